@@ -1,0 +1,164 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) dropless sparse Mixture-of-Experts
+ * feed-forward block.
+ *
+ * The block, for T tokens x[T,H], E routed experts of which k are used per
+ * token, and S always-on shared experts:
+ *
+ *   logits = x Wr^T + b                      moe_route    (router linear)
+ *   (idx, w) = top-k of logits, softmax      moe_route    (over the k selected)
+ *   group the T*k slots by expert            moe_permute  (stable, no drops)
+ *   h = SiLU(x Wg_e^T) * (x Wu_e^T)          moe_forward  (grouped GEMM 1)
+ *   o = s * w * (h Wd_e^T)                   moe_forward  (grouped GEMM 2)
+ *   y_t = sum_j o_(t,j) + sum_shared FFN(x_t) moe_combine (back to token order)
+ *
+ * Sources, by page and section:
+ *  - "PhiMoE in Transformers (Phi-3.5-MoE)", section 6: the router is a
+ *    bias-free nn.Linear hidden -> num_local_experts, followed (in eval mode)
+ *    by greedy top-1, masking, top-2 and a softmax over the selected experts;
+ *    section 2 item 3: the experts' gate and up projections are packed as
+ *    gate_up_proj (E, 2*I, H) and chunked into gate then up, act(gate) * up;
+ *    section 2 item 4: the block is dropless (no capacity factor, no padding).
+ *  - "Mixture of Experts in Transformers", expert backends: the grouped_mm
+ *    backend sorts and groups tokens by expert id and runs one grouped GEMM;
+ *    the runtime must dispatch tokens to their experts, run the projections,
+ *    apply the routing weights, then gather and reorder the results.
+ *    WeightConverter section: w1 (gate) and w3 (up) concatenated in that
+ *    order; down_proj stacked per expert (E, H, I).
+ *  - Instella-MoE modeling walk-through, FarSkipMoE and "config at a glance":
+ *    routed output times a scaling factor (2.5) plus always-on shared experts.
+ *  - GraniteMoeSWA page, decoder layer: the shared MLP output is added to the
+ *    sparse MoE output; shared experts are off when their width is 0.
+ *
+ * Conventions for every entry point:
+ *  - Every pointer argument except `shape` is a DEVICE pointer allocated and
+ *    owned by the caller; the library allocates no memory and keeps no state
+ *    beyond cached driver entry points and per-device attributes.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously; nothing synchronises the host.
+ *  - Arguments are validated on the host before any launch.  A failure returns
+ *    a status other than MOE_OK and enqueues nothing.  A launch failure
+ *    returns MOE_ERR_CUDA.  Faults that only the device can see (an expert
+ *    index out of range, a pipeline wait that times out) are OR-ed into the
+ *    caller's device word `err_flag` as MOE_ERR_* bit values (1 << status);
+ *    the caller zeroes it beforehand and reads it after synchronising.
+ *  - Layouts are row-major and dense.  moe_dtype selects float32 or bf16 for
+ *    x, the expert weights, the slot outputs and y.  The router weight and
+ *    bias and all routing weights are float32; indices are int32.
+ *  - The bf16 path needs H and I (and I_shared) to be multiples of 8 and all
+ *    device pointers 16-byte aligned; otherwise MOE_ERR_UNSUPPORTED.
+ *    E <= 256, k <= min(E, 16), n_shared <= 8, T*k < 2^31.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels implement */
+    MOE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    MOE_ERR_BAD_INDEX = 5,     /* device: an expert index outside [0, E) */
+    MOE_ERR_TIMEOUT = 6        /* device: a pipeline wait exceeded its limit */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef struct {
+    int64_t T;            /* tokens in this call (0 allowed: nothing is launched) */
+    int32_t H;            /* hidden size */
+    int32_t I;            /* routed expert intermediate size */
+    int32_t E;            /* routed experts */
+    int32_t k;            /* experts per token */
+    int32_t n_shared;     /* always-on shared experts (0 = none) */
+    int32_t I_shared;     /* shared expert intermediate size (0 when n_shared == 0) */
+    float routed_scale;   /* multiplies the routed sum (1.0 for plain top-k MoE) */
+    int32_t dtype;        /* moe_dtype of x, expert weights, y_slots and y */
+} moe_shape;
+
+/* Human-readable name of a status. Never NULL. */
+MOE_API const char* moe_status_str(moe_status status);
+
+/* Bytes of device workspace moe_permute and moe_forward need for `shape`
+ * (written to *bytes).  One buffer of this size serves both calls; its
+ * contents need no initialisation and are dead after each call returns on
+ * the stream. */
+MOE_API moe_status moe_workspace_size(const moe_shape* shape, size_t* bytes);
+
+/* Router and selection ("PhiMoE in Transformers", section 6).
+ *   x           [T, H]  dtype
+ *   w_router    [E, H]  float32 (nn.Linear layout: out x in)
+ *   router_bias [E]     float32, or NULL for a bias-free router
+ *   logits      [T, E]  float32 output, or NULL to skip writing it
+ *   topk_idx    [T, k]  int32 output: the k largest logits of each token in
+ *                       descending order; equal logits go to the lower index
+ *   topk_w      [T, k]  float32 output: softmax over the k selected logits
+ * Logits accumulate in float32. */
+MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const float* w_router,
+                     const float* router_bias, float* logits, int32_t* topk_idx,
+                     float* topk_w, void* stream);
+
+/* Dropless dispatch plan ("Mixture of Experts in Transformers", grouped_mm
+ * backend: sort and group tokens by expert id).  Slot q = t*k + j.
+ *   topk_idx  [T, k]  int32 input
+ *   counts    [E]     int32 output: slots routed to each expert (sum = T*k)
+ *   offsets   [E+1]   int32 output: exclusive prefix sum of counts
+ *   perm      [T*k]   int32 output: slot id at sorted position p, ordered by
+ *                     (expert ascending, slot id ascending) - deterministic
+ *   inv       [T*k]   int32 output: sorted position of slot q (perm^-1)
+ *   err_flag  [1]     int32, OR-ed with 1 << MOE_ERR_BAD_INDEX if an index is
+ *                     outside [0, E); such slots are skipped and the outputs
+ *                     are then unspecified (all writes stay in bounds)
+ *   workspace         at least moe_workspace_size() bytes */
+MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* err_flag,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* The expert FFNs, grouped by expert (two grouped GEMMs with fused epilogues).
+ *   x           [T, H]          dtype
+ *   offsets, perm               from moe_permute
+ *   topk_w      [T, k]          float32 routing weights from moe_route
+ *   gate_up     [E, 2I, H]      dtype; rows [0,I) gate, [I,2I) up
+ *   down        [E, H, I]       dtype
+ *   sh_gate_up  [S, 2Is, H]     dtype, or NULL when n_shared == 0
+ *   sh_down     [S, H, Is]      dtype, or NULL when n_shared == 0
+ *   y_slots     [T*k + S*T, H]  dtype output.  Row p < T*k holds
+ *               routed_scale * topk_w[perm[p]] * FFN_e(x_t) for slot perm[p]
+ *               (t = perm[p] / k, e its expert), rows in sorted order; row
+ *               T*k + s*T + t holds shared expert s applied to x_t (weight 1).
+ *   err_flag    [1] int32 device word (see conventions)
+ *   workspace   at least moe_workspace_size() bytes
+ * For small T*k the call streams each active expert's weights once (decode
+ * path); otherwise it runs the tensor-core grouped GEMMs. */
+MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* offsets,
+                       const int32_t* perm, const float* topk_w, const void* gate_up,
+                       const void* down, const void* sh_gate_up, const void* sh_down,
+                       void* y_slots, int32_t* err_flag, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Combine ("Mixture of Experts in Transformers", expert backends: gather and
+ * reorder the results).  y[t] = sum_j y_slots[inv[t*k+j]]
+ *                               + sum_s y_slots[T*k + s*T + t],
+ * summed in float32 and rounded once to dtype.
+ *   y_slots [T*k + S*T, H] dtype, inv [T*k] int32, y [T, H] dtype output. */
+MOE_API moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* inv,
+                       void* y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

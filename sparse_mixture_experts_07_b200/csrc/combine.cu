@@ -1,0 +1,114 @@
+// Combine: scatter the slot outputs back to token order and sum them.
+//
+// "Mixture of Experts in Transformers", expert backends: after the projections
+// and the routing weights, the runtime gathers and reorders the results into
+// token order.  y[t] = sum_j y_slots[inv[t*k+j]] + sum_s y_slots[T*k + s*T + t]
+// (shared experts: Instella-MoE walk-through, FarSkipMoE "routed + shared";
+// GraniteMoeSWA decoder layer, moe output + shared_mlp).  The sum is float32 in
+// a fixed order (j ascending, then s ascending) and is rounded once.
+//
+// One CTA of 256 threads per token row; each thread owns 16-byte vectors of
+// the row, so every y_slots row is read once, coalesced.  Memory-bound:
+// (k + S) * H * elem bytes read and H * elem bytes written per token.
+#include "common.cuh"
+
+namespace moe {
+
+template <typename T, int VEC>
+__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_slots,
+                                                      const int32_t* __restrict__ inv,
+                                                      T* __restrict__ y, int64_t n_tokens, int H,
+                                                      int k, int S) {
+    const int64_t routed_rows = n_tokens * k;
+    for (int64_t t = blockIdx.x; t < n_tokens; t += gridDim.x) {
+        int64_t rows[kMaxK + kMaxShared];
+        for (int j = 0; j < k; ++j) rows[j] = inv[t * k + j];
+        for (int s = 0; s < S; ++s) rows[k + s] = routed_rows + s * n_tokens + t;
+        for (int c = threadIdx.x * VEC; c < H; c += 256 * VEC) {
+            float acc[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+            for (int j = 0; j < k + S; ++j) {
+                const T* src = y_slots + rows[j] * H + c;
+                if constexpr (VEC == 8) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(src);
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        acc[2 * v] += bf16_to_f32(static_cast<uint16_t>(w[v] & 0xffffu));
+                        acc[2 * v + 1] += bf16_to_f32(static_cast<uint16_t>(w[v] >> 16));
+                    }
+                } else if constexpr (VEC == 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(src);
+                    acc[0] += u.x; acc[1] += u.y; acc[2] += u.z; acc[3] += u.w;
+                } else {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) acc[v] += ElemIO<T>::load(src, v);
+                }
+            }
+            T* dst = y + t * H + c;
+            if constexpr (VEC == 8) {
+                uint4 u;
+                u.x = pack_bf16x2(acc[0], acc[1]);
+                u.y = pack_bf16x2(acc[2], acc[3]);
+                u.z = pack_bf16x2(acc[4], acc[5]);
+                u.w = pack_bf16x2(acc[6], acc[7]);
+                *reinterpret_cast<uint4*>(dst) = u;
+            } else if constexpr (VEC == 4) {
+                *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            } else {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) ElemIO<T>::store(dst, v, acc[v]);
+            }
+        }
+    }
+}
+
+cudaError_t launch_combine(const moe_shape& s, const void* y_slots, const int32_t* inv, void* y,
+                           cudaStream_t st) {
+    const unsigned grid = static_cast<unsigned>(s.T < 1048576 ? s.T : 1048576);
+    if (s.dtype == MOE_BF16) {
+        combine_kernel<__nv_bfloat16, 8><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(y_slots), inv, static_cast<__nv_bfloat16*>(y), s.T,
+            s.H, s.k, s.n_shared);
+    } else if (s.H % 4 == 0) {
+        combine_kernel<float, 4><<<grid, 256, 0, st>>>(static_cast<const float*>(y_slots), inv,
+                                                       static_cast<float*>(y), s.T, s.H, s.k,
+                                                       s.n_shared);
+    } else {
+        combine_kernel<float, 1><<<grid, 256, 0, st>>>(static_cast<const float*>(y_slots), inv,
+                                                       static_cast<float*>(y), s.T, s.H, s.k,
+                                                       s.n_shared);
+    }
+    return cudaGetLastError();
+}
+
+// x_perm[p] = x[perm[p] / k]: the rows of x in sorted slot order (bf16, H % 8 == 0).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                          const int32_t* __restrict__ perm,
+                                                          uint4* __restrict__ x_perm, int64_t n_rows,
+                                                          int vec_per_row, int k) {
+    const int64_t total = n_rows * vec_per_row;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * 256) {
+        const int64_t p = i / vec_per_row;
+        const int v = static_cast<int>(i - p * vec_per_row);
+        const int64_t t = perm[p] / k;
+        x_perm[i] = x[t * vec_per_row + v];
+    }
+}
+
+cudaError_t launch_gather_rows(const moe_shape& s, const void* x, const int32_t* perm,
+                               void* x_perm, int num_sms, cudaStream_t st) {
+    const int64_t n_rows = s.T * s.k;
+    const int vpr = s.H / 8;
+    const int64_t total = n_rows * vpr;
+    int64_t grid = (total + 255) / 256;
+    if (grid > static_cast<int64_t>(num_sms) * 16) grid = static_cast<int64_t>(num_sms) * 16;
+    if (grid < 1) return cudaSuccess;
+    gather_rows_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
+        static_cast<const uint4*>(x), perm, static_cast<uint4*>(x_perm), n_rows, vpr, s.k);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

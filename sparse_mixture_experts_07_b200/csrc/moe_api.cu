@@ -1,0 +1,186 @@
+// The C ABI of include/moe.h: host-side validation, workspace layout and
+// dispatch to the kernels.  No memory is allocated here.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace moe {
+cudaError_t launch_route(const moe_shape&, const void*, const float*, const float*, float*,
+                         int32_t*, float*, cudaStream_t);
+size_t permute_workspace_bytes(const moe_shape&);
+cudaError_t launch_permute(const moe_shape&, const int32_t*, int32_t*, int32_t*, int32_t*,
+                           int32_t*, int32_t*, void*, cudaStream_t);
+cudaError_t launch_ffn_simt(const moe_shape&, const void*, const int32_t*, const int32_t*,
+                            const float*, const void*, const void*, const void*, const void*,
+                            void*, void*, void*, cudaStream_t);
+cudaError_t launch_ffn_sm100(const moe_shape&, const void*, const void*, const int32_t*,
+                             const int32_t*, const float*, const void*, const void*, const void*,
+                             const void*, void*, void*, void*, int32_t*, int, int, cudaStream_t);
+cudaError_t launch_combine(const moe_shape&, const void*, const int32_t*, void*, cudaStream_t);
+cudaError_t launch_gather_rows(const moe_shape&, const void*, const int32_t*, void*, int,
+                               cudaStream_t);
+}  // namespace moe
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+size_t elem_bytes(const moe_shape& s) { return s.dtype == MOE_BF16 ? 2 : 4; }
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    static int cached[64] = {0};
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
+    return n;
+}
+
+moe_status check_shape(const moe_shape* s) {
+    if (!s) return MOE_ERR_INVALID_ARG;
+    if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E <= 0 || s->k <= 0 || s->k > s->E ||
+        s->n_shared < 0 || (s->n_shared > 0 && s->I_shared <= 0) ||
+        (s->dtype != MOE_F32 && s->dtype != MOE_BF16))
+        return MOE_ERR_INVALID_ARG;
+    if (s->E > moe::kMaxExperts || s->k > moe::kMaxK || s->n_shared > moe::kMaxShared)
+        return MOE_ERR_UNSUPPORTED;
+    const int64_t rows = s->T * (s->k + s->n_shared);
+    if (s->T > (int64_t(1) << 31) || rows >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+    if (s->dtype == MOE_BF16) {
+        if (s->H % 8 || s->I % 8 || (s->n_shared > 0 && s->I_shared % 8))
+            return MOE_ERR_UNSUPPORTED;
+    }
+    return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+struct Workspace {
+    size_t permute_off, h_routed_off, h_shared_off, x_perm_off, total;
+};
+
+Workspace layout(const moe_shape& s) {
+    Workspace w{};
+    const size_t eb = elem_bytes(s);
+    const int64_t Tk = s.T * s.k;
+    size_t off = 0;
+    w.permute_off = off;
+    off += align_up(moe::permute_workspace_bytes(s));
+    w.h_routed_off = off;
+    off += align_up(static_cast<size_t>(Tk) * s.I * eb);
+    w.h_shared_off = off;
+    off += align_up(static_cast<size_t>(s.n_shared) * s.T * (s.n_shared ? s.I_shared : 0) * eb);
+    w.x_perm_off = off;
+    if (s.dtype == MOE_BF16) off += align_up(static_cast<size_t>(Tk) * s.H * 2);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_str(moe_status status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_BAD_INDEX: return "MOE_ERR_BAD_INDEX";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+moe_status moe_workspace_size(const moe_shape* shape, size_t* bytes) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = layout(*shape).total;
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_shape* shape, const void* x, const float* w_router,
+                     const float* router_bias, float* logits, int32_t* topk_idx, float* topk_w,
+                     void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_route(*shape, x, w_router, router_bias, logits, topk_idx,
+                                         topk_w, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* err_flag,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (shape->T > 0 && (!topk_idx || !perm || !inv)) return MOE_ERR_INVALID_ARG;
+    const Workspace w = layout(*shape);
+    if (w.total > 0 && (!workspace || workspace_bytes < w.total)) return MOE_ERR_WORKSPACE;
+    void* blk = static_cast<char*>(workspace) + w.permute_off;
+    return cuda_status(moe::launch_permute(*shape, topk_idx, counts, offsets, perm, inv, err_flag,
+                                           blk, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* offsets,
+                       const int32_t* perm, const float* topk_w, const void* gate_up,
+                       const void* down, const void* sh_gate_up, const void* sh_down,
+                       void* y_slots, int32_t* err_flag, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    const moe_shape& s = *shape;
+    if (s.T == 0) return MOE_OK;
+    if (!x || !offsets || !perm || !topk_w || !gate_up || !down || !y_slots)
+        return MOE_ERR_INVALID_ARG;
+    if (s.n_shared > 0 && (!sh_gate_up || !sh_down)) return MOE_ERR_INVALID_ARG;
+    const Workspace w = layout(s);
+    if (!workspace || workspace_bytes < w.total) return MOE_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    void* h_routed = ws + w.h_routed_off;
+    void* h_shared = ws + w.h_shared_off;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (s.dtype == MOE_F32) {
+        return cuda_status(moe::launch_ffn_simt(s, x, offsets, perm, topk_w, gate_up, down,
+                                                sh_gate_up, sh_down, h_routed, h_shared, y_slots,
+                                                cs));
+    }
+    const void* ptrs[] = {x, gate_up, down, y_slots, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
+    if (s.n_shared > 0 && (!aligned16(sh_gate_up) || !aligned16(sh_down)))
+        return MOE_ERR_UNSUPPORTED;
+    void* x_perm = ws + w.x_perm_off;
+    const int sms = num_sms();
+    cudaError_t e = moe::launch_gather_rows(s, x, perm, x_perm, sms, cs);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_ffn_sm100(s, x, x_perm, offsets, perm, topk_w, gate_up, down,
+                                             sh_gate_up, sh_down, h_routed, h_shared, y_slots,
+                                             err_flag, sms, 8, cs));
+}
+
+moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* inv, void* y,
+                       void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!y_slots || !inv || !y) return MOE_ERR_INVALID_ARG;
+    if (shape->dtype == MOE_BF16 && (!aligned16(y_slots) || !aligned16(y)))
+        return MOE_ERR_UNSUPPORTED;
+    if (shape->dtype == MOE_F32 && shape->H % 4 == 0 && (!aligned16(y_slots) || !aligned16(y)))
+        return MOE_ERR_UNSUPPORTED;
+    return cuda_status(
+        moe::launch_combine(*shape, y_slots, inv, y, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// Dropless dispatch plan: per-expert counts, offsets and the stable
+// permutation of the T*k slots by expert.
+//
+// "Mixture of Experts in Transformers", expert backends (grouped_mm): tokens
+// are sorted and grouped by expert id before one grouped GEMM; "PhiMoE in
+// Transformers", section 2 item 4: no token is dropped and there is no
+// capacity factor, so every slot gets a place.
+//
+// Three launches over blocks of 2048 consecutive slots:
+//   1. histogram: each block counts its slots per expert (shared-memory
+//      atomics; integer counts, so the result is order-independent);
+//   2. scan: one CTA turns the per-block counts into per-expert totals, the
+//      exclusive offsets, and each block's starting position per expert;
+//   3. scatter: each block ranks its slots stably (warp match + per-warp
+//      counts, rounds in slot order) and writes perm and inv.
+// The order (expert ascending, slot ascending) is fixed, so the plan is
+// bit-identical run to run.  Workspace: nblocks * E int32.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPermThreads = 256;
+constexpr int kPermRounds = 8;
+constexpr int kPermSlotsPerBlock = kPermThreads * kPermRounds;
+
+__global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(
+    const int32_t* __restrict__ idx, int64_t n, int E, int32_t* __restrict__ blk_counts,
+    int32_t* __restrict__ err_flag) {
+    __shared__ int32_t hist[kMaxExperts];
+    for (int e = threadIdx.x; e < E; e += kPermThreads) hist[e] = 0;
+    __syncthreads();
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermSlotsPerBlock;
+    bool bad = false;
+    for (int r = 0; r < kPermRounds; ++r) {
+        const int64_t q = base + r * kPermThreads + threadIdx.x;
+        if (q < n) {
+            const int e = idx[q];
+            if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+            else bad = true;
+        }
+    }
+    if (bad) raise_error(err_flag, MOE_ERR_BAD_INDEX);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kPermThreads)
+        blk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+// One CTA.  blk_counts [nblk][E] becomes blk_base [nblk][E] in place.
+__global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(
+    int32_t* __restrict__ blk, int nblk, int E, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets) {
+    __shared__ int32_t warp_sum[kPermThreads / 32];
+    const int e = threadIdx.x;
+    int32_t run = 0;
+    if (e < E) {
+        for (int b = 0; b < nblk; ++b) {
+            const int32_t c = blk[static_cast<int64_t>(b) * E + e];
+            blk[static_cast<int64_t>(b) * E + e] = run;
+            run += c;
+        }
+        counts[e] = run;
+    }
+    // exclusive scan of the per-expert totals (E <= 256 = blockDim)
+    const int lane = e & 31, warp = e >> 5;
+    int32_t v = (e < E) ? run : 0;
+    int32_t incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_sum[w];
+    const int32_t excl = before + incl - v;
+    if (e < E) {
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = excl + v;
+        for (int b = 0; b < nblk; ++b) blk[static_cast<int64_t>(b) * E + e] += excl;
+    }
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
+    const int32_t* __restrict__ idx, int64_t n, int E, const int32_t* __restrict__ blk_base,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+    __shared__ int32_t running[kMaxExperts];
+    __shared__ int32_t wcnt[kPermThreads / 32][kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += kPermThreads)
+        running[e] = blk_base[static_cast<int64_t>(blockIdx.x) * E + e];
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermSlotsPerBlock;
+    for (int r = 0; r < kPermRounds; ++r) {
+        for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads)
+            wcnt[i / E][i % E] = 0;
+        __syncthreads();
+        const int64_t q = base + r * kPermThreads + tid;
+        int e = -1;
+        if (q < n) {
+            e = idx[q];
+            if (e < 0 || e >= E) e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int lane_rank = __popc(peers & ((1u << lane) - 1u));
+        if (e >= 0 && lane_rank == 0) wcnt[warp][e] = __popc(peers);
+        __syncthreads();
+        if (e >= 0) {
+            int32_t p = running[e] + lane_rank;
+            for (int w = 0; w < warp; ++w) p += wcnt[w][e];
+            perm[p] = static_cast<int32_t>(q);
+            inv[q] = p;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += kPermThreads) {
+            int32_t s = 0;
+            for (int w = 0; w < kPermThreads / 32; ++w) s += wcnt[w][ee];
+            running[ee] += s;
+        }
+        __syncthreads();
+    }
+}
+
+size_t permute_workspace_bytes(const moe_shape& s) {
+    const int64_t n = s.T * s.k;
+    const int64_t nblk = (n + kPermSlotsPerBlock - 1) / kPermSlotsPerBlock;
+    return static_cast<size_t>(nblk) * s.E * sizeof(int32_t);
+}
+
+cudaError_t launch_permute(const moe_shape& s, const int32_t* idx, int32_t* counts,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* err_flag,
+                           void* workspace, cudaStream_t st) {
+    const int64_t n = s.T * s.k;
+    const int nblk = static_cast<int>((n + kPermSlotsPerBlock - 1) / kPermSlotsPerBlock);
+    int32_t* blk = static_cast<int32_t*>(workspace);
+    if (nblk > 0) {
+        permute_hist_kernel<<<nblk, kPermThreads, 0, st>>>(idx, n, s.E, blk, err_flag);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    permute_scan_kernel<<<1, kPermThreads, 0, st>>>(blk, nblk, s.E, counts, offsets);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || nblk == 0) return e;
+    permute_scatter_kernel<<<nblk, kPermThreads, 0, st>>>(idx, n, s.E, blk, perm, inv);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,156 @@
+// Router linear + top-k selection + softmax over the selected k, fused.
+//
+// "PhiMoE in Transformers (Phi-3.5-MoE)", section 6: the router is a bias-free
+// nn.Linear hidden -> num_local_experts; in eval mode the experts are chosen
+// greedily (top-1, mask it, take the next) and the chosen logits are soft-maxed.
+// The optional per-expert bias is added to the logits before selection.
+//
+// One CTA of 8 warps handles 32 tokens; warp w owns tokens 4w..4w+3 and lane l
+// owns experts l, l+32, ... (EPL per lane).  x and Wr are staged through shared
+// memory in chunks of 128 hidden columns; each lane accumulates its 4 x EPL
+// logits in float32, sequentially over h.  Selection runs as k rounds of a warp
+// arg-max (ties to the lower expert index) over the register-resident logits.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRouteTokens = 32;
+constexpr int kRouteHC = 128;              // hidden columns per chunk
+constexpr int kRouteLd = kRouteHC + 4;     // padded smem row (floats)
+
+template <typename T, int EPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(
+    const T* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
+    float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int64_t n_tokens, int H, int E, int k) {
+    extern __shared__ float4 smem_f4[];
+    float* xs = reinterpret_cast<float*>(smem_f4);          // [32][kRouteLd]
+    float* ws = xs + kRouteTokens * kRouteLd;               // [32*EPL][kRouteLd]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRouteTokens;
+    const int n_exp_rows = 32 * EPL;
+
+    float acc[4][EPL];
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) acc[t][j] = 0.f;
+
+    for (int h0 = 0; h0 < H; h0 += kRouteHC) {
+        const int hc = min(kRouteHC, H - h0);
+        __syncthreads();
+        for (int i = tid; i < kRouteTokens * kRouteHC; i += 256) {
+            int r = i / kRouteHC, c = i % kRouteHC;
+            int64_t tok = tok0 + r;
+            float v = 0.f;
+            if (tok < n_tokens && c < hc) v = ElemIO<T>::load(x, tok * H + h0 + c);
+            xs[r * kRouteLd + c] = v;
+        }
+        for (int i = tid; i < n_exp_rows * kRouteHC; i += 256) {
+            int r = i / kRouteHC, c = i % kRouteHC;
+            float v = 0.f;
+            if (r < E && c < hc) v = wr[static_cast<int64_t>(r) * H + h0 + c];
+            ws[r * kRouteLd + c] = v;
+        }
+        __syncthreads();
+        for (int c = 0; c < hc; c += 4) {
+            float4 xv[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                xv[t] = *reinterpret_cast<const float4*>(&xs[(warp * 4 + t) * kRouteLd + c]);
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                float4 wv = *reinterpret_cast<const float4*>(&ws[(lane + 32 * j) * kRouteLd + c]);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    acc[t][j] = fmaf(xv[t].x, wv.x, acc[t][j]);
+                    acc[t][j] = fmaf(xv[t].y, wv.y, acc[t][j]);
+                    acc[t][j] = fmaf(xv[t].z, wv.z, acc[t][j]);
+                    acc[t][j] = fmaf(xv[t].w, wv.w, acc[t][j]);
+                }
+            }
+        }
+    }
+
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int64_t tok = tok0 + warp * 4 + t;
+        if (tok >= n_tokens) continue;   // warp-uniform
+        float l[EPL];
+        unsigned taken = 0;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            l[j] = acc[t][j] + ((bias && e < E) ? bias[e] : 0.f);
+            if (logits && e < E) logits[tok * E + e] = l[j];
+        }
+        float sel_v[kMaxK];
+        int sel_e[kMaxK];
+        for (int r = 0; r < k; ++r) {
+            float best = -INFINITY;
+            int best_e = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const int e = lane + 32 * j;
+                if (e < E && !(taken >> j & 1u) && (l[j] > best || best_e == 0x7fffffff)) {
+                    best = l[j];
+                    best_e = e;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                float ov = __shfl_xor_sync(0xffffffffu, best, off);
+                int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
+                if (ov > best || (ov == best && oe < best_e)) {
+                    best = ov;
+                    best_e = oe;
+                }
+            }
+            if ((best_e & 31) == lane) taken |= 1u << (best_e >> 5);
+            sel_v[r] = best;
+            sel_e[r] = best_e;
+        }
+        if (lane == 0) {
+            // softmax over the selected logits; sel_v[0] is their maximum
+            float den = 0.f;
+            for (int r = 0; r < k; ++r) den += expf(sel_v[r] - sel_v[0]);
+            for (int r = 0; r < k; ++r) {
+                topk_idx[tok * k + r] = sel_e[r];
+                topk_w[tok * k + r] = expf(sel_v[r] - sel_v[0]) / den;
+            }
+        }
+    }
+}
+
+template <typename T, int EPL>
+static cudaError_t launch_route_t(const moe_shape& s, const void* x, const float* wr,
+                                  const float* bias, float* logits, int32_t* idx, float* w,
+                                  cudaStream_t st) {
+    const size_t smem = sizeof(float) * (kRouteTokens + 32 * EPL) * kRouteLd;
+    auto kern = route_topk_kernel<T, EPL>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    const int64_t blocks = (s.T + kRouteTokens - 1) / kRouteTokens;
+    kern<<<static_cast<unsigned>(blocks), 256, smem, st>>>(static_cast<const T*>(x), wr, bias,
+                                                           logits, idx, w, s.T, s.H, s.E, s.k);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route(const moe_shape& s, const void* x, const float* wr, const float* bias,
+                         float* logits, int32_t* idx, float* w, cudaStream_t st) {
+    const bool bf = s.dtype == MOE_BF16;
+    if (s.E <= 32)
+        return bf ? launch_route_t<__nv_bfloat16, 1>(s, x, wr, bias, logits, idx, w, st)
+                  : launch_route_t<float, 1>(s, x, wr, bias, logits, idx, w, st);
+    if (s.E <= 64)
+        return bf ? launch_route_t<__nv_bfloat16, 2>(s, x, wr, bias, logits, idx, w, st)
+                  : launch_route_t<float, 2>(s, x, wr, bias, logits, idx, w, st);
+    if (s.E <= 128)
+        return bf ? launch_route_t<__nv_bfloat16, 4>(s, x, wr, bias, logits, idx, w, st)
+                  : launch_route_t<float, 4>(s, x, wr, bias, logits, idx, w, st);
+    return bf ? launch_route_t<__nv_bfloat16, 8>(s, x, wr, bias, logits, idx, w, st)
+              : launch_route_t<float, 8>(s, x, wr, bias, logits, idx, w, st);
+}
+
+}  // namespace moe

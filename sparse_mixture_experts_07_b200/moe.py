@@ -1,0 +1,218 @@
+"""Python binding of include/moe.h (ctypes).
+
+Argument marshalling only: every step of the block runs in libmoe.so's CUDA
+kernels.  PyTorch provides device memory and the current stream.  If the
+library has not been built, every call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_INDEX", 6: "MOE_ERR_TIMEOUT"}
+EXPORTS = ("moe_status_str", "moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
+           "moe_combine")
+
+
+class MoEShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("I_shared", ctypes.c_int32), ("routed_scale", ctypes.c_float),
+                ("dtype", ctypes.c_int32)]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libmoe.so (raises if it is missing: build it with
+    `python -m sparse_mixture_experts_07_b200.build`)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libmoe.so is not built ({path}); run "
+                           "`python -m sparse_mixture_experts_07_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, S = ctypes.c_void_p, ctypes.POINTER(MoEShape)
+    lib.moe_status_str.argtypes = [ctypes.c_int]
+    lib.moe_status_str.restype = ctypes.c_char_p
+    lib.moe_workspace_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
+    lib.moe_route.argtypes = [S, P, P, P, P, P, P, P]
+    lib.moe_permute.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.moe_combine.argtypes = [S, P, P, P, P]
+    for f in EXPORTS[1:]:
+        getattr(lib, f).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise MoEError(rc, where)
+
+
+@dataclass(frozen=True)
+class Shape:
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    n_shared: int = 0
+    I_shared: int = 0
+    routed_scale: float = 1.0
+    dtype: int = MOE_BF16
+
+    @staticmethod
+    def from_config(cfg) -> "Shape":
+        return Shape(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.n_shared, cfg.I_shared,
+                     cfg.routed_scale, MOE_BF16 if cfg.dtype == "bf16" else MOE_F32)
+
+    def c(self) -> MoEShape:
+        return MoEShape(self.T, self.H, self.I, self.E, self.k, self.n_shared, self.I_shared,
+                        self.routed_scale, self.dtype)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == MOE_BF16 else torch.float32
+
+    @property
+    def slot_rows(self) -> int:
+        return self.T * (self.k + self.n_shared)
+
+
+def workspace_size(shape: Shape) -> int:
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    _check(lib.moe_workspace_size(ctypes.byref(shape.c()), ctypes.byref(n)), "moe_workspace_size")
+    return n.value
+
+
+def alloc_workspace(shape: Shape, device="cuda") -> torch.Tensor:
+    return torch.empty(max(workspace_size(shape), 1), dtype=torch.uint8, device=device)
+
+
+def route(shape: Shape, x, w_router, router_bias=None, logits=False, out=None, stream=None):
+    """(topk_idx [T,k] int32, topk_w [T,k] f32, logits [T,E] f32 or None)."""
+    lib = load_library()
+    dev = x.device
+    idx = out["topk_idx"] if out else torch.empty(shape.T, shape.k, dtype=torch.int32, device=dev)
+    w = out["topk_w"] if out else torch.empty(shape.T, shape.k, dtype=torch.float32, device=dev)
+    lg = torch.empty(shape.T, shape.E, dtype=torch.float32, device=dev) if logits else None
+    _check(lib.moe_route(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(router_bias),
+                         _ptr(lg), _ptr(idx), _ptr(w), _stream(stream)), "moe_route")
+    return idx, w, lg
+
+
+def permute(shape: Shape, topk_idx, workspace, err_flag, out=None, stream=None):
+    """(counts [E], offsets [E+1], perm [T*k], inv [T*k]) int32."""
+    lib = load_library()
+    dev = topk_idx.device
+    n = shape.T * shape.k
+    if out:
+        counts, offsets, perm, inv = out["counts"], out["offsets"], out["perm"], out["inv"]
+    else:
+        counts = torch.empty(shape.E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(shape.E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(n, dtype=torch.int32, device=dev)
+        inv = torch.empty(n, dtype=torch.int32, device=dev)
+    _check(lib.moe_permute(ctypes.byref(shape.c()), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                           _ptr(perm), _ptr(inv), _ptr(err_flag), _ptr(workspace),
+                           workspace.numel(), _stream(stream)), "moe_permute")
+    return counts, offsets, perm, inv
+
+
+def forward(shape: Shape, x, offsets, perm, topk_w, gate_up, down, sh_gate_up, sh_down,
+            workspace, err_flag, y_slots=None, stream=None):
+    """y_slots [T*k + S*T, H] (dtype): weighted expert outputs in sorted slot order,
+    then the shared experts' outputs."""
+    lib = load_library()
+    if y_slots is None:
+        y_slots = torch.empty(shape.slot_rows, shape.H, dtype=shape.torch_dtype, device=x.device)
+    _check(lib.moe_forward(ctypes.byref(shape.c()), _ptr(x), _ptr(offsets), _ptr(perm),
+                           _ptr(topk_w), _ptr(gate_up), _ptr(down), _ptr(sh_gate_up),
+                           _ptr(sh_down), _ptr(y_slots), _ptr(err_flag), _ptr(workspace),
+                           workspace.numel(), _stream(stream)), "moe_forward")
+    return y_slots
+
+
+def combine(shape: Shape, y_slots, inv, y=None, stream=None):
+    """y [T, H] (dtype)."""
+    lib = load_library()
+    if y is None:
+        y = torch.empty(shape.T, shape.H, dtype=shape.torch_dtype, device=y_slots.device)
+    _check(lib.moe_combine(ctypes.byref(shape.c()), _ptr(y_slots), _ptr(inv), _ptr(y),
+                           _stream(stream)), "moe_combine")
+    return y
+
+
+class MoELayer:
+    """The whole block on one device: route -> permute -> forward -> combine.
+
+    Holds the weights (device tensors) and a reusable workspace; `__call__`
+    takes x [T, H] on the device and returns y [T, H].  Intermediates of the
+    last call are kept in `self.last` for inspection.
+    """
+
+    def __init__(self, shape: Shape, w_router, router_bias, gate_up, down, sh_gate_up=None,
+                 sh_down=None):
+        self.shape = shape
+        self.w_router, self.router_bias = w_router, router_bias
+        self.gate_up, self.down = gate_up, down
+        self.sh_gate_up, self.sh_down = sh_gate_up, sh_down
+        dev = gate_up.device
+        self.workspace = alloc_workspace(shape, dev)
+        self.err_flag = torch.zeros(1, dtype=torch.int32, device=dev)
+        T, k, E, H = shape.T, shape.k, shape.E, shape.H
+        self.buf = {
+            "topk_idx": torch.empty(T, k, dtype=torch.int32, device=dev),
+            "topk_w": torch.empty(T, k, dtype=torch.float32, device=dev),
+            "counts": torch.empty(E, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+            "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
+            "inv": torch.empty(T * k, dtype=torch.int32, device=dev),
+            "y_slots": torch.empty(shape.slot_rows, H, dtype=shape.torch_dtype, device=dev),
+            "y": torch.empty(T, H, dtype=shape.torch_dtype, device=dev),
+        }
+        self.last = None
+
+    def __call__(self, x, stream=None, y=None):
+        s, b = self.shape, self.buf
+        idx, w, _ = route(s, x, self.w_router, self.router_bias, out=b, stream=stream)
+        counts, offsets, perm, inv = permute(s, idx, self.workspace, self.err_flag, out=b,
+                                             stream=stream)
+        forward(s, x, offsets, perm, w, self.gate_up, self.down, self.sh_gate_up, self.sh_down,
+                self.workspace, self.err_flag, y_slots=b["y_slots"], stream=stream)
+        out = combine(s, b["y_slots"], inv, y=b["y"] if y is None else y, stream=stream)
+        self.last = b
+        return out
+
+    def device_error(self) -> int:
+        """Device-detected error bits (synchronises)."""
+        return int(self.err_flag.item())

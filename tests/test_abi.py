@@ -1,0 +1,132 @@
+"""The C ABI: the library builds, loads, exports every declared entry point, and
+rejects bad arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_07_b200 as moe
+from sparse_mixture_experts_07_b200 import build as moe_build
+from sparse_mixture_experts_07_b200.moe import MoEShape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.load_library()
+
+
+def declared_entry_points():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", text)
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for n in ("moe_route", "moe_permute", "moe_forward", "moe_combine", "moe_workspace_size",
+              "moe_status_str"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_entry_points():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in moe.moe.STATUS.items():
+        assert lib.moe_status_str(code).decode() == name
+    assert lib.moe_status_str(99).decode() == "MOE_ERR_UNKNOWN"
+
+
+def _shape(**kw):
+    base = dict(T=64, H=128, I=256, E=8, k=2, n_shared=0, I_shared=0, routed_scale=1.0,
+                dtype=moe.MOE_BF16)
+    base.update(kw)
+    return MoEShape(**base)
+
+
+def _ws(lib, s):
+    n = ctypes.c_size_t(0)
+    rc = lib.moe_workspace_size(ctypes.byref(s), ctypes.byref(n))
+    return rc, n.value
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(k=9), 1), (dict(k=0), 1), (dict(E=0), 1), (dict(T=-1), 1), (dict(H=0), 1),
+    (dict(n_shared=1, I_shared=0), 1), (dict(dtype=7), 1),
+    (dict(E=300, k=2), 2), (dict(k=17, E=64), 2), (dict(n_shared=9, I_shared=64), 2),
+    (dict(H=100), 2), (dict(I=100), 2), (dict(n_shared=1, I_shared=36), 2),
+    (dict(H=100, dtype=moe.MOE_F32), 0), (dict(T=0), 0),
+])
+def test_shape_validation(lib, kw, expected):
+    rc, _ = _ws(lib, _shape(**kw))
+    assert rc == expected
+
+
+def test_workspace_size_grows_with_tokens(lib):
+    sizes = [_ws(lib, _shape(T=t))[1] for t in (1, 64, 1000, 4096)]
+    assert sizes == sorted(sizes) and sizes[0] > 0
+    _, with_shared = _ws(lib, _shape(n_shared=2, I_shared=128))
+    assert with_shared > _ws(lib, _shape())[1]
+
+
+def test_null_pointers_rejected_before_launch(lib):
+    s = _shape()
+    p = ctypes.c_void_p(16)   # never dereferenced: validation fails first
+    assert lib.moe_route(ctypes.byref(s), None, p, None, None, p, p, None) == 1
+    assert lib.moe_route(ctypes.byref(s), p, None, None, None, p, p, None) == 1
+    assert lib.moe_permute(ctypes.byref(s), p, None, p, p, p, None, p, 1 << 30, None) == 1
+    assert lib.moe_forward(ctypes.byref(s), p, p, p, p, None, p, None, None, p, None, p,
+                           1 << 30, None) == 1
+    sh = _shape(n_shared=2, I_shared=128)
+    assert lib.moe_forward(ctypes.byref(sh), p, p, p, p, p, p, None, None, p, None, p,
+                           1 << 30, None) == 1
+    assert lib.moe_combine(ctypes.byref(s), None, p, p, None) == 1
+    assert lib.moe_route(None, p, p, None, None, p, p, None) == 1
+
+
+def test_small_workspace_rejected(lib):
+    s = _shape()
+    rc, need = _ws(lib, s)
+    p = ctypes.c_void_p(256)
+    assert lib.moe_permute(ctypes.byref(s), p, p, p, p, p, None, p, need - 1, None) == 3
+    assert lib.moe_permute(ctypes.byref(s), p, p, p, p, p, None, None, need, None) == 3
+    assert lib.moe_forward(ctypes.byref(s), p, p, p, p, p, p, None, None, p, None, p,
+                           need - 1, None) == 3
+
+
+def test_misaligned_bf16_pointers_rejected(lib):
+    s = _shape()
+    _, need = _ws(lib, s)
+    ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 2)
+    assert lib.moe_forward(ctypes.byref(s), bad, ok, ok, ok, ok, ok, None, None, ok, None, ok,
+                           need, None) == 2
+    assert lib.moe_combine(ctypes.byref(s), bad, ok, ok, None) == 2
+
+
+def test_zero_tokens_is_a_no_op(lib):
+    s = _shape(T=0)
+    assert lib.moe_route(ctypes.byref(s), None, None, None, None, None, None, None) == 0
+    assert lib.moe_forward(ctypes.byref(s), None, None, None, None, None, None, None, None,
+                           None, None, None, 0, None) == 0
+    assert lib.moe_combine(ctypes.byref(s), None, None, None, None) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    import importlib
+    m = importlib.import_module("sparse_mixture_experts_07_b200.moe")
+    saved = m._lib
+    m._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="not built"):
+            m.load_library(str(tmp_path / "libmoe.so"))
+    finally:
+        m._lib = saved

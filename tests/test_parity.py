@@ -1,0 +1,112 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Routing indices, counts, offsets and the permutation are
+compared bit-exactly; outputs by relative L2 error (1e-5 float32, 1e-2 bf16).
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity_util import (check_outputs, check_routing, run_gpu, sample_tokens, to_device)
+from sparse_mixture_experts_07_b200.inputs import CONFIGS, MoEConfig, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+# Small shapes the oracle finishes in seconds; each spans several tiles and has
+# ragged tails in rows (experts' counts), in N and in K.
+SMALL = [
+    MoEConfig("f32_small", T=200, H=136, I=200, E=8, k=2, dtype="f32"),
+    MoEConfig("f32_shared", T=77, H=64, I=96, E=6, k=3, n_shared=2, I_shared=40,
+              routed_scale=2.5, dtype="f32", zipf_s=1.0),
+    MoEConfig("bf16_tiles", T=300, H=512, I=384, E=8, k=2),
+    MoEConfig("bf16_ragged", T=333, H=712, I=328, E=8, k=2),
+    MoEConfig("bf16_many_experts", T=256, H=256, I=136, E=64, k=6, n_shared=2, I_shared=128,
+              routed_scale=2.5, zipf_s=1.2),
+    MoEConfig("bf16_gptoss_like", T=512, H=360, I=360, E=32, k=4, zipf_s=1.0),
+    MoEConfig("bf16_empty_experts", T=5, H=256, I=128, E=16, k=1),
+    MoEConfig("bf16_one_token", T=1, H=512, I=256, E=16, k=2),
+    MoEConfig("bf16_k_equals_E", T=40, H=128, I=128, E=4, k=4),
+]
+
+
+def _run(cfg, weights_device="cuda"):
+    inp = make_inputs(cfg, seed=0, weights_device="cpu")
+    res = run_gpu(cfg, to_device(inp))
+    return inp, res
+
+
+def test_tiny_config_full_parity(cuda_ok):
+    cfg = CONFIGS["tiny"]
+    inp, res = _run(cfg)
+    assert res["err"] == 0
+    check_routing(cfg, inp, res)
+    err = check_outputs(cfg, inp, res)
+    assert err < 1e-5
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_small_configs(cuda_ok, cfg):
+    inp, res = _run(cfg)
+    assert res["err"] == 0
+    check_routing(cfg, inp, res)
+    check_outputs(cfg, inp, res)
+
+
+def test_routed_slot_rows_hold_weighted_expert_outputs(cuda_ok):
+    # y_slots row p = routed_scale * w * FFN_e(x_t) for slot perm[p]
+    import oracle
+    cfg = MoEConfig("slots", T=64, H=256, I=256, E=8, k=2, n_shared=1, I_shared=128,
+                    routed_scale=2.5)
+    inp, res = _run(cfg)
+    perm = res["perm"].numpy()
+    ys = res["y_slots"].float().numpy()
+    w = res["topk_w"].numpy().reshape(-1)
+    idx = res["topk_idx"].numpy().reshape(-1)
+    for p in (0, 5, 63, 100, cfg.T * cfg.k - 1):
+        q = perm[p]
+        t, e = q // cfg.k, idx[q]
+        ref = cfg.routed_scale * w[q] * oracle.expert(inp["gate_up"][e], inp["down"][e],
+                                                      inp["x"][t].double().numpy())
+        assert np.linalg.norm(ys[p] - ref) <= 1e-2 * np.linalg.norm(ref)
+    for t in (0, 31, 63):
+        ref = oracle.expert(inp["sh_gate_up"][0], inp["sh_down"][0], inp["x"][t].double().numpy())
+        row = ys[cfg.T * cfg.k + t]
+        assert np.linalg.norm(row - ref) <= 1e-2 * np.linalg.norm(ref)
+
+
+def test_repeat_runs_are_bit_identical(cuda_ok):
+    cfg = MoEConfig("det", T=1000, H=256, I=256, E=16, k=4, zipf_s=1.0)
+    inp = to_device(make_inputs(cfg))
+    a = run_gpu(cfg, inp)
+    b = run_gpu(cfg, inp)
+    for key in ("topk_idx", "perm", "y"):
+        assert torch.equal(a[key], b[key])
+
+
+def test_bad_expert_index_sets_error_flag(cuda_ok):
+    import sparse_mixture_experts_07_b200 as moe
+    shape = moe.Shape(T=8, H=128, I=128, E=4, k=2)
+    idx = torch.tensor([[0, 1]] * 7 + [[2, 9]], dtype=torch.int32, device="cuda")
+    ws = moe.alloc_workspace(shape)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    counts, offsets, perm, inv = moe.permute(shape, idx, ws, err)
+    torch.cuda.synchronize()
+    assert err.item() == 1 << 5
+    assert int(counts.sum()) == 15
+
+
+FULL = ["mixtral", "phimoe_prefill", "gptoss", "dsv3", "phimoe_decode1", "phimoe_decode8",
+        "phimoe_decode64"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(cuda_ok, name):
+    """Full-size configurations: routing for every token, the plan's
+    invariants, and the outputs of a sample of tokens against the oracle."""
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg, seed=0, weights_device="cuda")
+    res = run_gpu(cfg, to_device(inp))
+    assert res["err"] == 0
+    host = {key: (v.cpu() if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
+    toks = sample_tokens(cfg.T, 24 if cfg.T > 64 else cfg.T)
+    check_routing(cfg, host, res)
+    check_outputs(cfg, host, res, tokens=toks)
