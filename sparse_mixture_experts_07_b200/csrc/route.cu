@@ -8,7 +8,7 @@
 // One CTA of 8 warps handles 32 tokens; warp w owns tokens 4w..4w+3 and lane l
 // owns experts l, l+32, ... (EPL per lane).  x and Wr are staged through shared
 // memory in chunks of 128 hidden columns; each lane accumulates its 4 x EPL
-// logits in float32, sequentially over h.  Selection runs as k rounds of a warp
+// logits in float32, sequentially within a chunk, then chunk by chunk.  Selection runs as k rounds of a warp
 // arg-max (ties to the lower expert index) over the register-resident logits.
 #include "common.cuh"
 
@@ -53,6 +53,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
             ws[r * kRouteLd + c] = v;
         }
         __syncthreads();
+        // per-chunk partial sums keep the float32 rounding error near
+        // (sqrt(128) + sqrt(H/128)) ulp instead of sqrt(H) ulp
+        float part[4][EPL];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) part[t][j] = 0.f;
         for (int c = 0; c < hc; c += 4) {
             float4 xv[4];
 #pragma unroll
@@ -63,13 +70,17 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
                 float4 wv = *reinterpret_cast<const float4*>(&ws[(lane + 32 * j) * kRouteLd + c]);
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    acc[t][j] = fmaf(xv[t].x, wv.x, acc[t][j]);
-                    acc[t][j] = fmaf(xv[t].y, wv.y, acc[t][j]);
-                    acc[t][j] = fmaf(xv[t].z, wv.z, acc[t][j]);
-                    acc[t][j] = fmaf(xv[t].w, wv.w, acc[t][j]);
+                    part[t][j] = fmaf(xv[t].x, wv.x, part[t][j]);
+                    part[t][j] = fmaf(xv[t].y, wv.y, part[t][j]);
+                    part[t][j] = fmaf(xv[t].z, wv.z, part[t][j]);
+                    part[t][j] = fmaf(xv[t].w, wv.w, part[t][j]);
                 }
             }
         }
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) acc[t][j] += part[t][j];
     }
 
 #pragma unroll

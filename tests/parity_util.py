@@ -11,7 +11,11 @@ from sparse_mixture_experts_07_b200.inputs import MoEConfig, make_inputs
 
 BF16_TOL = 1e-2     # relative L2 error bound for bf16 configurations
 F32_TOL = 1e-5      # relative L2 error bound for float32 configurations
-W_TOL = 1e-6        # routing weights, absolute
+# Router logits accumulate H products in float32 (partial sums of 128); their
+# absolute error stays far below 2e-5 for |x| ~ 1, |Wr| ~ 0.02, H <= 4096.
+LOGIT_TOL = 2e-5
+# Softmax over the selected k: |dw_i| <= w_i (|dl_i| + sum_j w_j |dl_j|) <= 2 max|dl|.
+W_TOL = 2 * LOGIT_TOL
 
 
 def to_device(inp: dict, dev="cuda") -> dict:
@@ -57,8 +61,10 @@ def check_routing(cfg: MoEConfig, inp: dict, res: dict, tokens=None):
     g_w = res["topk_w"].numpy()
     sel = slice(None) if tokens is None else np.asarray(tokens)
     assert np.array_equal(g_idx[sel], o_idx), "routing indices differ"
-    assert np.abs(g_w[sel] - o_w).max() <= W_TOL
-    assert np.abs(res["logits"].numpy()[sel] - lg).max() < 1e-4
+    lerr = float(np.abs(res["logits"].numpy()[sel] - lg).max())
+    werr = float(np.abs(g_w[sel] - o_w).max())
+    assert lerr <= LOGIT_TOL, f"logit error {lerr:.3e}"
+    assert werr <= W_TOL, f"routing weight error {werr:.3e}"
     if tokens is None:
         counts, offsets, perm, inv = oracle.permute(o_idx, E)
         assert np.array_equal(res["counts"].numpy(), counts)
