@@ -207,9 +207,12 @@ def count_launches(step_fn) -> int:
     """Kernels of libmoe.so launched by one step (CUPTI via torch.profiler)."""
     from torch.profiler import ProfilerActivity, profile
     torch.cuda.synchronize()
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        step_fn()
-        torch.cuda.synchronize()
+    try:
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step_fn()
+            torch.cuda.synchronize()
+    except Exception:       # CUPTI unavailable (e.g. under another profiler)
+        return -1
     n = 0
     for ev in prof.events():
         name = ev.name or ""
@@ -330,7 +333,7 @@ def run_cuda(args, cfg, rank, local, world):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * cfg.H * eb,
                 "d2h_bytes_per_step": cfg.T * cfg.H * eb},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * args.steps if launches_per_step >= 0 else None,
         "clocks": clk.summary(),
         "expert_counts": counts.tolist(),
     }
