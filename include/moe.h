@@ -127,6 +127,24 @@ MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, 
                        int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* err_flag,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_permute for callers that cannot allocate device memory: for example a
+ * plugin whose host framework owns every device allocation and hands it only
+ * its input and output buffers, or a latency-critical path where a cudaMalloc,
+ * which may synchronise the device, is not allowed.  The pages have no
+ * counterpart: this is a packaging of moe_permute, not a step of the method.
+ * Arguments, outputs and errors are those of moe_permute, without the
+ * workspace.  Its scratch (the per-block expert counts) is a 1 MiB array in
+ * the library's static device memory, which every GPU that loads the library
+ * holds until the process exits; shapes needing more than that,
+ * ceil(T*k / 2048) * E > 262144, return MOE_ERR_UNSUPPORTED.  The first call
+ * on a device looks up that array's device address (cudaGetSymbolAddress) and
+ * caches it; make that first call before any stream capture.  All calls share
+ * the one array, so calls that can overlap on the GPU (unordered streams)
+ * race on it.  Nothing in it needs clearing between calls. */
+MOE_API moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_idx,
+                                       int32_t* counts, int32_t* offsets, int32_t* perm,
+                                       int32_t* inv, int32_t* err_flag, void* stream);
+
 /* The expert FFNs, grouped by expert (two grouped GEMMs with fused epilogues).
  *   x           [T, H]          dtype
  *   offsets, perm               from moe_permute

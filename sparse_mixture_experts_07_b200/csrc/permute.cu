@@ -145,3 +145,76 @@ cudaError_t launch_permute(const moe_shape& s, const int32_t* idx, int32_t* coun
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: the same dispatch plan for callers that cannot allocate
+// device memory - for example a plugin whose host framework owns every device
+// allocation and hands it only its input and output buffers, or a latency-
+// critical path where a cudaMalloc (which may synchronise the device) is not
+// allowed.  The per-block expert counts live in a file-scope __device__ array
+// of kNoallocScratchInts int32 (1 MiB); every GPU that loads this library holds
+// it until the process exits.
+//
+// Host code must not pass `g_permute_scratch` itself to a kernel: on the host
+// that name is only a stand-in, not a device address.  The device address is
+// looked up once per device with cudaGetSymbolAddress, on the first call made
+// while that device is current, and cached; make that first call before any
+// stream capture.  The array keeps the last call's contents; the histogram
+// kernel overwrites every entry it later reads, so nothing needs clearing.
+// All calls share the one array: calls whose kernels may overlap on the GPU
+// (different streams without ordering between them) race on it.
+#include <mutex>
+
+namespace moe {
+constexpr int64_t kNoallocScratchInts = 256 * 1024;
+constexpr int kNoallocMaxDevices = 64;
+}  // namespace moe
+
+static __device__ __align__(256) int32_t g_permute_scratch[moe::kNoallocScratchInts];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[moe::kNoallocMaxDevices] = {nullptr};
+
+// Device address of g_permute_scratch on the current device (looked up once).
+cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= moe::kNoallocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_permute_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_idx,
+                                          int32_t* counts, int32_t* offsets, int32_t* perm,
+                                          int32_t* inv, int32_t* err_flag, void* stream) {
+    if (!shape) return MOE_ERR_INVALID_ARG;
+    const moe_shape& s = *shape;
+    if (s.T < 0 || s.H <= 0 || s.I <= 0 || s.E <= 0 || s.k <= 0 || s.k > s.E ||
+        s.n_shared < 0 || (s.n_shared > 0 && s.I_shared <= 0) ||
+        (s.dtype != MOE_F32 && s.dtype != MOE_BF16))
+        return MOE_ERR_INVALID_ARG;
+    if (s.E > moe::kMaxExperts || s.k > moe::kMaxK || s.T * s.k >= (int64_t(1) << 31))
+        return MOE_ERR_UNSUPPORTED;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (s.T > 0 && (!topk_idx || !perm || !inv)) return MOE_ERR_INVALID_ARG;
+    // the plan needs ceil(T*k / 2048) * E ints of scratch
+    if (moe::permute_workspace_bytes(s) > sizeof(int32_t) * moe::kNoallocScratchInts)
+        return MOE_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t e = moe::launch_permute(s, topk_idx, counts, offsets, perm, inv, err_flag, scratch,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
