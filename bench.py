@@ -253,7 +253,8 @@ def run_cuda(args, cfg, rank, local, world):
     with ClockSampler(local) as clk:
         s0.record(stream)
         for i in range(args.steps):
-            idx, w, _ = moe.route(shape, x, layer.w_router, layer.router_bias, out=b)
+            idx, w, _ = moe.route(shape, x, layer.w_router, layer.router_bias, out=b,
+                                  err_flag=layer.err_flag)
             moe.permute(shape, idx, layer.workspace, layer.err_flag, out=b)
             fwd_start[i].record(stream)
             moe.forward(shape, x, b["offsets"], b["perm"], w, layer.gate_up, layer.down,
@@ -310,10 +311,15 @@ def run_cuda(args, cfg, rank, local, world):
     else:
         flops = 2.0 * cfg.T * (3 * cfg.k * cfg.H * cfg.I + 3 * cfg.n_shared * cfg.I_shared * cfg.H)
         achieved = flops / (fwd_ms / 1000.0) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+        # a timed region of back-to-back GEMMs longer than ~0.25 s runs into the
+        # power cap: compare with the sustained GEMM figure, else the burst one
+        long_run = ms_total / 1000.0 >= 0.25 and peaks["bf16_tflops_sustained"]
+        peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                 "kernel": "moe_forward (gather + grouped GEMM gate_up/SwiGLU + grouped GEMM down)",
-                "peak_kind": f"{peaks['source']} bf16 burst"}
+                "peak_kind": f"{peaks['source']} bf16 {'sustained' if long_run else 'burst'}",
+                "frac_of_burst": achieved / peaks["bf16_tflops"]}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -352,8 +358,8 @@ def run_cuda(args, cfg, rank, local, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -106,10 +106,14 @@ MOE_API moe_status moe_workspace_size(const moe_shape* shape, size_t* bytes);
  *   topk_idx    [T, k]  int32 output: the k largest logits of each token in
  *                       descending order; equal logits go to the lower index
  *   topk_w      [T, k]  float32 output: softmax over the k selected logits
- * Logits accumulate in float32. */
+ *   err_flag    [1]     int32 device word, or NULL (see conventions)
+ * Logits accumulate in float32.  Up to 256 tokens run one CTA per token on the
+ * CUDA cores; more tokens with bf16 x and E <= 64 run on the tensor cores,
+ * the float32 weight split into three bf16 terms (exact to one float32 ulp);
+ * anything else runs on the CUDA cores. */
 MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const float* w_router,
-                     const float* router_bias, float* logits, int32_t* topk_idx,
-                     float* topk_w, void* stream);
+                             const float* router_bias, float* logits, int32_t* topk_idx,
+                             float* topk_w, int32_t* err_flag, void* stream);
 
 /* Dropless dispatch plan ("Mixture of Experts in Transformers", grouped_mm
  * backend: sort and group tokens by expert id).  Slot q = t*k + j.

@@ -7,6 +7,10 @@
 namespace moe {
 cudaError_t launch_route(const moe_shape&, const void*, const float*, const float*, float*,
                          int32_t*, float*, cudaStream_t);
+cudaError_t launch_route_tc(const moe_shape&, const void*, const float*, const float*, float*,
+                            int32_t*, float*, int32_t*, cudaStream_t);
+cudaError_t launch_route_small(const moe_shape&, const void*, const float*, const float*, float*,
+                               int32_t*, float*, cudaStream_t);
 size_t permute_workspace_bytes(const moe_shape&);
 cudaError_t launch_permute(const moe_shape&, const int32_t*, int32_t*, int32_t*, int32_t*,
                            int32_t*, int32_t*, void*, cudaStream_t);
@@ -16,6 +20,9 @@ cudaError_t launch_ffn_simt(const moe_shape&, const void*, const int32_t*, const
 cudaError_t launch_ffn_sm100(const moe_shape&, const void*, const void*, const int32_t*,
                              const int32_t*, const float*, const void*, const void*, const void*,
                              const void*, void*, void*, void*, int32_t*, int, int, cudaStream_t);
+cudaError_t launch_ffn_decode(const moe_shape&, const void*, const int32_t*, const int32_t*,
+                              const float*, const void*, const void*, const void*, const void*,
+                              void*, void*, void*, int, cudaStream_t);
 cudaError_t launch_combine(const moe_shape&, const void*, const int32_t*, void*, cudaStream_t);
 cudaError_t launch_gather_rows(const moe_shape&, const void*, const int32_t*, void*, int,
                                cudaStream_t);
@@ -109,13 +116,21 @@ moe_status moe_workspace_size(const moe_shape* shape, size_t* bytes) {
 
 moe_status moe_route(const moe_shape* shape, const void* x, const float* w_router,
                      const float* router_bias, float* logits, int32_t* topk_idx, float* topk_w,
-                     void* stream) {
+                     int32_t* err_flag, void* stream) {
     moe_status st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
     if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // few tokens: one CTA per token; many tokens, bf16: tensor cores; else CUDA cores
+    if (shape->T <= 256 && shape->H <= 32768 && aligned16(w_router))
+        return cuda_status(moe::launch_route_small(*shape, x, w_router, router_bias, logits,
+                                                   topk_idx, topk_w, cs));
+    if (shape->dtype == MOE_BF16 && shape->E <= 64 && aligned16(x) && aligned16(w_router))
+        return cuda_status(moe::launch_route_tc(*shape, x, w_router, router_bias, logits,
+                                                topk_idx, topk_w, err_flag, cs));
     return cuda_status(moe::launch_route(*shape, x, w_router, router_bias, logits, topk_idx,
-                                         topk_w, static_cast<cudaStream_t>(stream)));
+                                         topk_w, cs));
 }
 
 moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
@@ -160,8 +175,13 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* off
         if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
     if (s.n_shared > 0 && (!aligned16(sh_gate_up) || !aligned16(sh_down)))
         return MOE_ERR_UNSUPPORTED;
-    void* x_perm = ws + w.x_perm_off;
     const int sms = num_sms();
+    // decode batches (<= 8 rows per expert): stream the active experts' weights
+    if (s.T <= 8)
+        return cuda_status(moe::launch_ffn_decode(s, x, offsets, perm, topk_w, gate_up, down,
+                                                  sh_gate_up, sh_down, h_routed, h_shared,
+                                                  y_slots, sms, cs));
+    void* x_perm = ws + w.x_perm_off;
     cudaError_t e = moe::launch_gather_rows(s, x, perm, x_perm, sms, cs);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     return cuda_status(moe::launch_ffn_sm100(s, x, x_perm, offsets, perm, topk_w, gate_up, down,

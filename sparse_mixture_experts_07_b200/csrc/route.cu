@@ -133,6 +133,120 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     }
 }
 
+// Few tokens (decode): one CTA per token, 8 warps over the experts.  The token
+// row is staged in shared memory as float32; warp w computes the logits of
+// experts w, w+8, ...: each lane reads 4 consecutive weights per step (16-byte
+// loads, 8 steps unrolled so many loads are in flight), then the warp sums the
+// lane partials with a butterfly.  Warp 0 then selects as above.
+template <typename T>
+__global__ void __launch_bounds__(256) route_small_kernel(
+    const T* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
+    float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int H, int E, int k) {
+    extern __shared__ float4 smem_f4[];
+    float* xs = reinterpret_cast<float*>(smem_f4);     // [H]
+    float* lg = xs + ((H + 3) & ~3);                   // [E]
+    const int64_t tok = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int h = tid; h < H; h += 256) xs[h] = ElemIO<T>::load(x, tok * H + h);
+    __syncthreads();
+    const bool vec = (H % 4) == 0;
+    for (int e = warp; e < E; e += 8) {
+        const float* w = wr + static_cast<int64_t>(e) * H;
+        float acc = 0.f;
+        if (vec) {
+            const int n4 = H >> 2;
+            int i = lane;
+            for (; i + 7 * 32 < n4; i += 8 * 32) {
+                float4 wv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) wv[u] = __ldg(reinterpret_cast<const float4*>(w) + i + u * 32);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float4 xv = *reinterpret_cast<const float4*>(&xs[4 * (i + u * 32)]);
+                    acc = fmaf(wv[u].x, xv.x, acc);
+                    acc = fmaf(wv[u].y, xv.y, acc);
+                    acc = fmaf(wv[u].z, xv.z, acc);
+                    acc = fmaf(wv[u].w, xv.w, acc);
+                }
+            }
+            for (; i < n4; i += 32) {
+                const float4 wv = __ldg(reinterpret_cast<const float4*>(w) + i);
+                const float4 xv = *reinterpret_cast<const float4*>(&xs[4 * i]);
+                acc = fmaf(wv.x, xv.x, acc);
+                acc = fmaf(wv.y, xv.y, acc);
+                acc = fmaf(wv.z, xv.z, acc);
+                acc = fmaf(wv.w, xv.w, acc);
+            }
+        } else {
+            for (int h = lane; h < H; h += 32) acc = fmaf(w[h], xs[h], acc);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) lg[e] = acc + (bias ? bias[e] : 0.f);
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    if (logits)
+        for (int e = lane; e < E; e += 32) logits[tok * E + e] = lg[e];
+    float sel_v[kMaxK];
+    int sel_e[kMaxK];
+    for (int r = 0; r < k; ++r) {
+        float best = -INFINITY;
+        int best_e = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            bool taken = false;
+            for (int q = 0; q < r; ++q) taken |= (sel_e[q] == e);
+            if (!taken && (lg[e] > best || best_e == 0x7fffffff)) {
+                best = lg[e];
+                best_e = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
+            if (ov > best || (ov == best && oe < best_e)) {
+                best = ov;
+                best_e = oe;
+            }
+        }
+        sel_v[r] = best;
+        sel_e[r] = best_e;
+    }
+    if (lane == 0) {
+        float den = 0.f;
+        for (int r = 0; r < k; ++r) den += expf(sel_v[r] - sel_v[0]);
+        for (int r = 0; r < k; ++r) {
+            topk_idx[tok * k + r] = sel_e[r];
+            topk_w[tok * k + r] = expf(sel_v[r] - sel_v[0]) / den;
+        }
+    }
+}
+
+cudaError_t launch_route_small(const moe_shape& s, const void* x, const float* wr,
+                               const float* bias, float* logits, int32_t* idx, float* w,
+                               cudaStream_t st) {
+    const size_t smem = sizeof(float) * (((s.H + 3) & ~3) + s.E);
+    if (smem > 200 * 1024) return cudaErrorInvalidValue;
+    if (s.dtype == MOE_BF16) {
+        auto kern = route_small_kernel<__nv_bfloat16>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        kern<<<static_cast<unsigned>(s.T), 256, smem, st>>>(
+            static_cast<const __nv_bfloat16*>(x), wr, bias, logits, idx, w, s.H, s.E, s.k);
+    } else {
+        auto kern = route_small_kernel<float>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        kern<<<static_cast<unsigned>(s.T), 256, smem, st>>>(static_cast<const float*>(x), wr,
+                                                            bias, logits, idx, w, s.H, s.E, s.k);
+    }
+    return cudaGetLastError();
+}
+
 template <typename T, int EPL>
 static cudaError_t launch_route_t(const moe_shape& s, const void* x, const float* wr,
                                   const float* bias, float* logits, int32_t* idx, float* w,

@@ -53,7 +53,7 @@ def load_library(path: str = LIB_PATH):
     lib.moe_status_str.argtypes = [ctypes.c_int]
     lib.moe_status_str.restype = ctypes.c_char_p
     lib.moe_workspace_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
-    lib.moe_route.argtypes = [S, P, P, P, P, P, P, P]
+    lib.moe_route.argtypes = [S, P, P, P, P, P, P, P, P]
     lib.moe_permute.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_combine.argtypes = [S, P, P, P, P]
@@ -118,7 +118,8 @@ def alloc_workspace(shape: Shape, device="cuda") -> torch.Tensor:
     return torch.empty(max(workspace_size(shape), 1), dtype=torch.uint8, device=device)
 
 
-def route(shape: Shape, x, w_router, router_bias=None, logits=False, out=None, stream=None):
+def route(shape: Shape, x, w_router, router_bias=None, logits=False, out=None, stream=None,
+          err_flag=None):
     """(topk_idx [T,k] int32, topk_w [T,k] f32, logits [T,E] f32 or None)."""
     lib = load_library()
     dev = x.device
@@ -126,7 +127,8 @@ def route(shape: Shape, x, w_router, router_bias=None, logits=False, out=None, s
     w = out["topk_w"] if out else torch.empty(shape.T, shape.k, dtype=torch.float32, device=dev)
     lg = torch.empty(shape.T, shape.E, dtype=torch.float32, device=dev) if logits else None
     _check(lib.moe_route(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(router_bias),
-                         _ptr(lg), _ptr(idx), _ptr(w), _stream(stream)), "moe_route")
+                         _ptr(lg), _ptr(idx), _ptr(w), _ptr(err_flag), _stream(stream)),
+           "moe_route")
     return idx, w, lg
 
 
@@ -204,7 +206,8 @@ class MoELayer:
 
     def __call__(self, x, stream=None, y=None):
         s, b = self.shape, self.buf
-        idx, w, _ = route(s, x, self.w_router, self.router_bias, out=b, stream=stream)
+        idx, w, _ = route(s, x, self.w_router, self.router_bias, out=b, stream=stream,
+                          err_flag=self.err_flag)
         counts, offsets, perm, inv = permute(s, idx, self.workspace, self.err_flag, out=b,
                                              stream=stream)
         forward(s, x, offsets, perm, w, self.gate_up, self.down, self.sh_gate_up, self.sh_down,

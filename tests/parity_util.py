@@ -11,11 +11,20 @@ from sparse_mixture_experts_07_b200.inputs import MoEConfig, make_inputs
 
 BF16_TOL = 1e-2     # relative L2 error bound for bf16 configurations
 F32_TOL = 1e-5      # relative L2 error bound for float32 configurations
-# Router logits accumulate H products in float32 (partial sums of 128); their
-# absolute error stays far below 2e-5 for |x| ~ 1, |Wr| ~ 0.02, H <= 4096.
-LOGIT_TOL = 2e-5
+
+
+def logit_tol(H: int, logits: np.ndarray) -> float:
+    """Bound on the router's float32 logit error.
+
+    The products x_h * w_h are exact on either router (bf16 x times the three
+    bf16 terms of w, or float32 FMA).  The sum is float32: on the tensor cores
+    the running sum is rounded once per 16-product MMA step, so H/16 roundings
+    of at most 2^-23 of |logit| each; the CUDA-core router does fewer.  Twice
+    that, plus 1e-6 for the weight split and the bias add."""
+    return 2.0 * (H / 16.0) * 2.0 ** -23 * float(np.abs(logits).max()) + 1e-6
+
+
 # Softmax over the selected k: |dw_i| <= w_i (|dl_i| + sum_j w_j |dl_j|) <= 2 max|dl|.
-W_TOL = 2 * LOGIT_TOL
 
 
 def to_device(inp: dict, dev="cuda") -> dict:
@@ -63,8 +72,10 @@ def check_routing(cfg: MoEConfig, inp: dict, res: dict, tokens=None):
     assert np.array_equal(g_idx[sel], o_idx), "routing indices differ"
     lerr = float(np.abs(res["logits"].numpy()[sel] - lg).max())
     werr = float(np.abs(g_w[sel] - o_w).max())
-    assert lerr <= LOGIT_TOL, f"logit error {lerr:.3e}"
-    assert werr <= W_TOL, f"routing weight error {werr:.3e}"
+    ltol = logit_tol(cfg.H, lg)
+    assert lerr <= ltol, f"logit error {lerr:.3e} > {ltol:.3e}"
+    assert werr <= 2 * ltol, f"routing weight error {werr:.3e} > {2 * ltol:.3e}"
+    print(f"[{cfg.name}] logit error {lerr:.2e} (bound {ltol:.2e}), weight error {werr:.2e}")
     if tokens is None:
         counts, offsets, perm, inv = oracle.permute(o_idx, E)
         assert np.array_equal(res["counts"].numpy(), counts)
@@ -92,6 +103,7 @@ def check_outputs(cfg: MoEConfig, inp: dict, res: dict, tokens=None):
         y_g = y_g[np.asarray(tokens)]
     err = rel_l2(y_g.astype(np.float64), y_o)
     assert err <= tolerance(cfg), f"relative L2 error {err:.3e} > {tolerance(cfg)}"
+    print(f"[{cfg.name}] output relative L2 error {err:.2e} (bound {tolerance(cfg)})")
     return err
 
 

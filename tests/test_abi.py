@@ -81,8 +81,8 @@ def test_workspace_size_grows_with_tokens(lib):
 def test_null_pointers_rejected_before_launch(lib):
     s = _shape()
     p = ctypes.c_void_p(16)   # never dereferenced: validation fails first
-    assert lib.moe_route(ctypes.byref(s), None, p, None, None, p, p, None) == 1
-    assert lib.moe_route(ctypes.byref(s), p, None, None, None, p, p, None) == 1
+    assert lib.moe_route(ctypes.byref(s), None, p, None, None, p, p, None, None) == 1
+    assert lib.moe_route(ctypes.byref(s), p, None, None, None, p, p, None, None) == 1
     assert lib.moe_permute(ctypes.byref(s), p, None, p, p, p, None, p, 1 << 30, None) == 1
     assert lib.moe_forward(ctypes.byref(s), p, p, p, p, None, p, None, None, p, None, p,
                            1 << 30, None) == 1
@@ -90,7 +90,7 @@ def test_null_pointers_rejected_before_launch(lib):
     assert lib.moe_forward(ctypes.byref(sh), p, p, p, p, p, p, None, None, p, None, p,
                            1 << 30, None) == 1
     assert lib.moe_combine(ctypes.byref(s), None, p, p, None) == 1
-    assert lib.moe_route(None, p, p, None, None, p, p, None) == 1
+    assert lib.moe_route(None, p, p, None, None, p, p, None, None) == 1
 
 
 def test_small_workspace_rejected(lib):
@@ -114,7 +114,7 @@ def test_misaligned_bf16_pointers_rejected(lib):
 
 def test_zero_tokens_is_a_no_op(lib):
     s = _shape(T=0)
-    assert lib.moe_route(ctypes.byref(s), None, None, None, None, None, None, None) == 0
+    assert lib.moe_route(ctypes.byref(s), None, None, None, None, None, None, None, None) == 0
     assert lib.moe_forward(ctypes.byref(s), None, None, None, None, None, None, None, None,
                            None, None, None, 0, None) == 0
     assert lib.moe_combine(ctypes.byref(s), None, None, None, None) == 0

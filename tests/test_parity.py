@@ -25,6 +25,15 @@ SMALL = [
     MoEConfig("bf16_empty_experts", T=5, H=256, I=128, E=16, k=1),
     MoEConfig("bf16_one_token", T=1, H=512, I=256, E=16, k=2),
     MoEConfig("bf16_k_equals_E", T=40, H=128, I=128, E=4, k=4),
+    # > 256 tokens: tensor-core router (E <= 64) or CUDA-core tiled router
+    MoEConfig("f32_many_tokens", T=600, H=72, I=64, E=8, k=2, dtype="f32"),
+    MoEConfig("bf16_E128", T=300, H=128, I=64, E=128, k=4),
+    MoEConfig("bf16_router_tc_E40", T=520, H=200, I=64, E=40, k=3, zipf_s=1.0),
+    # decode batches (T <= 8) take the weight-streaming path; ragged H, I, Is
+    MoEConfig("bf16_decode_shared", T=7, H=712, I=328, E=16, k=3, n_shared=2, I_shared=200,
+              routed_scale=2.5),
+    MoEConfig("bf16_decode_T8", T=8, H=1024, I=512, E=4, k=4),
+    MoEConfig("bf16_just_above_decode", T=9, H=256, I=256, E=8, k=2),
 ]
 
 
