@@ -179,6 +179,14 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const int3
 MOE_API moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* inv,
                        void* y, void* stream);
 
+/* Diagnostic with no counterpart in the pages: runs the bounded pipeline wait
+ * that every kernel here uses on an mbarrier nothing ever arrives on, so that
+ * it expires after timeout_ns (0 < timeout_ns <= 10 s).  The kernel then ORs
+ * 1 << MOE_ERR_TIMEOUT into the device word err_flag (required) and returns;
+ * the context stays usable.  Lets a caller check the device-side failure
+ * path without a fault. */
+MOE_API moe_status moe_selftest_wait_timeout(int64_t timeout_ns, int32_t* err_flag, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

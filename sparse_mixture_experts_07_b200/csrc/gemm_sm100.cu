@@ -32,7 +32,7 @@
 // Every wait is bounded by a deadline on %globaltimer; on expiry the kernel
 // sets MOE_ERR_TIMEOUT in err_flag, leaves its loops, drains its MMAs and
 // frees its tensor memory.
-#include "common.cuh"
+#include "gemm_common.cuh"
 
 namespace moe {
 
@@ -49,55 +49,6 @@ constexpr int TMEM_COLS = 512;                // two 256-column accumulators
 constexpr int THREADS = 192;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 }  // namespace sm100
-
-enum : int { kSwiGLU = 0, kScaled = 1 };
-
-struct GemmParams {
-    const int32_t* offsets;   // [E+1]
-    const int32_t* perm;      // [T*k]
-    const float* topk_w;      // [T*k]
-    int64_t T;
-    int E, S, k;
-    int n_tiles_routed, n_tiles_shared;
-    int K_routed, K_shared;          // contraction length
-    int N_routed, N_shared;          // valid output columns
-    int b_rows_routed, b_rows_shared;  // B rows per expert (2I / H)
-    int half_routed, half_shared;      // kSwiGLU: offset of the up rows (I / Is)
-    void* out_routed;
-    void* out_shared;
-    int64_t ld_routed, ld_shared;      // output row strides (elements)
-    int64_t out_row0_shared;           // kScaled: first y_slots row of shared outputs
-    float routed_scale;
-    int group_m;
-    int32_t* err_flag;
-    uint64_t timeout_ns;
-};
-
-struct TileCoord {
-    int g;          // group
-    int m0;         // first row within the group
-    int n0;         // first output column
-    int rows;       // rows of the group
-    bool routed;
-};
-
-__device__ __forceinline__ TileCoord decode_tile(const GroupTable& gt, const GemmParams& p,
-                                                 int tile, int n_cols_per_tile) {
-    TileCoord c;
-    c.g = find_group(gt, tile);
-    c.routed = c.g < p.E;
-    c.rows = gt.rows[c.g];
-    const int local = tile - gt.tile_start[c.g];
-    const int nt = c.routed ? p.n_tiles_routed : p.n_tiles_shared;
-    const int mt = (c.rows + sm100::BM - 1) / sm100::BM;
-    const int band = local / (p.group_m * nt);
-    const int within = local - band * p.group_m * nt;
-    const int m_base = band * p.group_m;
-    const int gm = min(p.group_m, mt - m_base);
-    c.n0 = (within / gm) * n_cols_per_tile;
-    c.m0 = (m_base + within % gm) * sm100::BM;
-    return c;
-}
 
 template <int EPI>
 __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
@@ -161,7 +112,7 @@ __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile);
+                const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, BM);
                 const CUtensorMap* ma = c.routed ? &map_a_routed : &map_a_shared;
                 const CUtensorMap* mb = c.routed ? &map_b_routed : &map_b_shared;
                 const int K = c.routed ? p.K_routed : p.K_shared;
@@ -204,7 +155,7 @@ __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile);
+                const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, BM);
                 const int K = c.routed ? p.K_routed : p.K_shared;
                 const int num_kb = (K + BK - 1) / BK;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, deadline)) { ok = false; break; }
@@ -244,7 +195,7 @@ __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile);
+            const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, BM);
             if (!mbar_wait(&tfull[acc], acc_phase, deadline)) {
                 raise_error(p.err_flag, MOE_ERR_TIMEOUT);
                 break;
@@ -326,48 +277,6 @@ __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
-
-// ---------------------------------------------------------------------------
-// Host side: tensor maps and launches.
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// 2D bf16 row-major [rows, cols], box = 64 columns x box_rows rows, 128-byte swizzle.
-static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
-                     int box_rows) {
-    EncodeTiledFn enc = get_encode_fn();
-    if (!enc || rows <= 0 || cols <= 0) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(sm100::BK), static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-struct GemmLaunchInfo {
-    int grid;
-};
-
-static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // GEMM 1 (gate_up + SwiGLU) and GEMM 2 (down + weight) for the bf16 path.
 cudaError_t launch_ffn_sm100(const moe_shape& s, const void* x, const void* x_perm,

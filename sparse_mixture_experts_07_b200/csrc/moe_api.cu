@@ -23,6 +23,10 @@ cudaError_t launch_ffn_sm100(const moe_shape&, const void*, const void*, const i
 cudaError_t launch_ffn_decode(const moe_shape&, const void*, const int32_t*, const int32_t*,
                               const float*, const void*, const void*, const void*, const void*,
                               void*, void*, void*, int, cudaStream_t);
+cudaError_t launch_ffn_sm100_pair(const moe_shape&, const void*, const void*, const int32_t*,
+                                  const int32_t*, const float*, const void*, const void*,
+                                  const void*, const void*, void*, void*, void*, int32_t*, int, int,
+                                  cudaStream_t);
 cudaError_t launch_combine(const moe_shape&, const void*, const int32_t*, void*, cudaStream_t);
 cudaError_t launch_gather_rows(const moe_shape&, const void*, const int32_t*, void*, int,
                                cudaStream_t);
@@ -184,6 +188,13 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* off
     void* x_perm = ws + w.x_perm_off;
     cudaError_t e = moe::launch_gather_rows(s, x, perm, x_perm, sms, cs);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+#ifndef MOE_GEMM_PAIR
+#define MOE_GEMM_PAIR 1
+#endif
+    if (MOE_GEMM_PAIR)
+        return cuda_status(moe::launch_ffn_sm100_pair(s, x, x_perm, offsets, perm, topk_w, gate_up,
+                                                      down, sh_gate_up, sh_down, h_routed,
+                                                      h_shared, y_slots, err_flag, sms, 4, cs));
     return cuda_status(moe::launch_ffn_sm100(s, x, x_perm, offsets, perm, topk_w, gate_up, down,
                                              sh_gate_up, sh_down, h_routed, h_shared, y_slots,
                                              err_flag, sms, 8, cs));

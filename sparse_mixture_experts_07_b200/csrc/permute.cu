@@ -14,7 +14,8 @@
 //   3. scatter: each block ranks its slots stably (warp match + per-warp
 //      counts, rounds in slot order) and writes perm and inv.
 // The order (expert ascending, slot ascending) is fixed, so the plan is
-// bit-identical run to run.  Workspace: nblocks * E int32.
+// bit-identical run to run.  Workspace: nblocks * E int32.  A plan of a
+// single block (T*k <= 2048) runs all three steps in one CTA and one launch.
 #include "common.cuh"
 
 namespace moe {
@@ -120,6 +121,79 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
     }
 }
 
+// Plans of at most one block of slots (T*k <= 2048, e.g. decode batches): the
+// three steps above in one CTA and one launch, no workspace.
+__global__ void __launch_bounds__(kPermThreads) permute_single_kernel(
+    const int32_t* __restrict__ idx, int64_t n, int E, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    int32_t* __restrict__ err_flag) {
+    __shared__ int32_t hist[kMaxExperts];
+    __shared__ int32_t running[kMaxExperts];
+    __shared__ int32_t wcnt[kPermThreads / 32][kMaxExperts];
+    __shared__ int32_t warp_sum[kPermThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += kPermThreads) hist[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int r = 0; r < kPermRounds; ++r) {
+        const int64_t q = r * kPermThreads + tid;
+        if (q < n) {
+            const int e = idx[q];
+            if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+            else bad = true;
+        }
+    }
+    if (bad) raise_error(err_flag, MOE_ERR_BAD_INDEX);
+    __syncthreads();
+    // exclusive scan of the counts (E <= 256 = blockDim)
+    const int32_t v = tid < E ? hist[tid] : 0;
+    int32_t incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_sum[w];
+    if (tid < E) {
+        const int32_t excl = before + incl - v;
+        counts[tid] = v;
+        offsets[tid] = excl;
+        running[tid] = excl;
+        if (tid == E - 1) offsets[E] = excl + v;
+    }
+    // stable scatter, rounds in slot order (as permute_scatter_kernel)
+    for (int r = 0; r < kPermRounds; ++r) {
+        for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads) wcnt[i / E][i % E] = 0;
+        __syncthreads();
+        const int64_t q = r * kPermThreads + tid;
+        int e = -1;
+        if (q < n) {
+            e = idx[q];
+            if (e < 0 || e >= E) e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int lane_rank = __popc(peers & ((1u << lane) - 1u));
+        if (e >= 0 && lane_rank == 0) wcnt[warp][e] = __popc(peers);
+        __syncthreads();
+        if (e >= 0) {
+            int32_t p = running[e] + lane_rank;
+            for (int w = 0; w < warp; ++w) p += wcnt[w][e];
+            perm[p] = static_cast<int32_t>(q);
+            inv[q] = p;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += kPermThreads) {
+            int32_t s = 0;
+            for (int w = 0; w < kPermThreads / 32; ++w) s += wcnt[w][ee];
+            running[ee] += s;
+        }
+        __syncthreads();
+    }
+}
+
 size_t permute_workspace_bytes(const moe_shape& s) {
     const int64_t n = s.T * s.k;
     const int64_t nblk = (n + kPermSlotsPerBlock - 1) / kPermSlotsPerBlock;
@@ -131,6 +205,11 @@ cudaError_t launch_permute(const moe_shape& s, const int32_t* idx, int32_t* coun
                            void* workspace, cudaStream_t st) {
     const int64_t n = s.T * s.k;
     const int nblk = static_cast<int>((n + kPermSlotsPerBlock - 1) / kPermSlotsPerBlock);
+    if (nblk == 1) {
+        permute_single_kernel<<<1, kPermThreads, 0, st>>>(idx, n, s.E, counts, offsets, perm, inv,
+                                                          err_flag);
+        return cudaGetLastError();
+    }
     int32_t* blk = static_cast<int32_t*>(workspace);
     if (nblk > 0) {
         permute_hist_kernel<<<nblk, kPermThreads, 0, st>>>(idx, n, s.E, blk, err_flag);

@@ -119,3 +119,24 @@ def test_full_size_sampled(cuda_ok, name):
     toks = sample_tokens(cfg.T, 24 if cfg.T > 64 else cfg.T)
     check_routing(cfg, host, res)
     check_outputs(cfg, host, res, tokens=toks)
+
+
+def test_bounded_wait_expires_and_reports_timeout(cuda_ok):
+    """A pipeline wait that nothing satisfies expires, reports MOE_ERR_TIMEOUT
+    in the device error word, and leaves the context usable."""
+    import ctypes
+    import sparse_mixture_experts_07_b200 as moe
+    lib = moe.load_library()
+    f = lib.moe_selftest_wait_timeout
+    f.argtypes = [ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert f(0, ctypes.c_void_p(err.data_ptr()), stream) == 1
+    assert f(20_000_000, ctypes.c_void_p(err.data_ptr()), stream) == 0
+    torch.cuda.synchronize()
+    assert err.item() == 1 << 6
+    cfg = MoEConfig("after_timeout", T=32, H=128, I=128, E=4, k=2)
+    inp, res = _run(cfg)
+    assert res["err"] == 0
+    check_routing(cfg, inp, res)
