@@ -13,7 +13,12 @@
 //     CTA alone issues tcgen05.mma.cta_group::2 (M=256, N=256, K=16) and its
 //     commits arrive on both CTAs' barriers (stage free, accumulator full);
 //   - each CTA's epilogue reads its own 128 TMEM lanes (= its 128 rows) and
-//     reports the accumulator free on the even CTA's barrier.
+//     reports the accumulator free on the even CTA's barrier;
+//   - the last m-tile of a group with at most 128 real rows runs as an M=128
+//     pair MMA (64 rows per CTA), which the hardware stores folded: TMEM lanes
+//     0-63 hold the first half of the columns, lanes 64-127 the second half.
+//     For GEMM 1 each CTA then loads 64 gate rows and the matching 64 up rows,
+//     so every lane still holds gate and up of the same output columns.
 // No TMA multicast is used: each CTA fetches its own operand halves.
 // Waits are bounded as in the one-CTA kernel.
 #include "gemm_common.cuh"
@@ -38,11 +43,22 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint16_t BOTH = 0x3;                // cluster ranks 0 and 1
 }  // namespace pair
 
+// Tile of the pair kernel.  The last m-tile of a group is a "half" tile when
+// at most 128 of its rows are real: it runs as an M=128 pair MMA (64 rows per
+// CTA) instead of M=256, which halves the padding of that tile.
+__device__ __forceinline__ TileCoord decode_pair_tile(const GroupTable& gt, const GemmParams& p,
+                                                      int tile, int n_cols_per_tile, bool& half) {
+    const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, pair::BM);
+    half = c.rows - c.m0 <= pair::BM / 2;
+    return c;
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
     const __grid_constant__ CUtensorMap map_a_routed, const __grid_constant__ CUtensorMap map_a_shared,
     const __grid_constant__ CUtensorMap map_b_routed, const __grid_constant__ CUtensorMap map_b_shared,
-    const GemmParams p) {
+    const __grid_constant__ CUtensorMap map_bh_routed,
+    const __grid_constant__ CUtensorMap map_bh_shared, const GemmParams p) {
     using namespace pair;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ GroupTable gt;
@@ -104,19 +120,26 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = cluster; tile < total && ok; tile += n_clusters) {
-                const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, BM);
+                bool half;
+                const TileCoord c = decode_pair_tile(gt, p, tile, n_cols_per_tile, half);
                 const CUtensorMap* ma = c.routed ? &map_a_routed : &map_a_shared;
                 const CUtensorMap* mb = c.routed ? &map_b_routed : &map_b_shared;
+                const CUtensorMap* mbh = c.routed ? &map_bh_routed : &map_bh_shared;
                 const int K = c.routed ? p.K_routed : p.K_shared;
                 const int eidx = c.routed ? c.g : c.g - p.E;
-                // this CTA's 128 A rows: routed -> sorted slot rows; shared GEMM 1 ->
-                // token rows; shared GEMM 2 -> that expert's block of h
-                int a_row = gt.row0[c.g] + c.m0 + static_cast<int>(rank) * BM_CTA;
-                if (EPI == kSwiGLU && !c.routed) a_row = c.m0 + static_cast<int>(rank) * BM_CTA;
-                // this CTA's 128 B rows: GEMM 1 gate (rank 0) or up (rank 1); GEMM 2 half
+                const int up_off = c.routed ? p.half_routed : p.half_shared;
+                // this CTA's A rows (128 of a full tile, the first 64 used of a half
+                // tile): routed -> sorted slot rows; shared GEMM 1 -> token rows;
+                // shared GEMM 2 -> that expert's block of h
+                const int rows_cta = half ? BM_CTA / 2 : BM_CTA;
+                int a_row = gt.row0[c.g] + c.m0 + static_cast<int>(rank) * rows_cta;
+                if (EPI == kSwiGLU && !c.routed) a_row = c.m0 + static_cast<int>(rank) * rows_cta;
+                // this CTA's 128 B rows.  GEMM 1, full tile: gate (rank 0) or up
+                // (rank 1) of the 128 columns; GEMM 1, half tile: 64 gate rows then
+                // the matching 64 up rows of columns n0 + 64 rank; GEMM 2: its half
                 const int b_rows = c.routed ? p.b_rows_routed : p.b_rows_shared;
                 int b_row = eidx * b_rows + c.n0;
-                if (EPI == kSwiGLU) b_row += rank ? (c.routed ? p.half_routed : p.half_shared) : 0;
+                if (EPI == kSwiGLU) b_row += half ? static_cast<int>(rank) * 64 : (rank ? up_off : 0);
                 else b_row += static_cast<int>(rank) * BN_CTA;
                 const int num_kb = (K + BK - 1) / BK;
                 for (int kb = 0; kb < num_kb; ++kb) {
@@ -125,7 +148,12 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const uint32_t bar = full_leader + stage * 8;
                     tma_load_2d_pair(sa, ma, bar, kb * BK, a_row);
-                    tma_load_2d_pair(sa + A_BYTES, mb, bar, kb * BK, b_row);
+                    if (EPI == kSwiGLU && half) {
+                        tma_load_2d_pair(sa + A_BYTES, mbh, bar, kb * BK, b_row);
+                        tma_load_2d_pair(sa + A_BYTES + B_BYTES / 2, mbh, bar, kb * BK, b_row + up_off);
+                    } else {
+                        tma_load_2d_pair(sa + A_BYTES, mb, bar, kb * BK, b_row);
+                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -134,14 +162,17 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA (even CTA)
         if (lane == 0 && leader) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            constexpr uint32_t idesc_full = idesc_bf16_f32(BM, BN);
+            constexpr uint32_t idesc_half = idesc_bf16_f32(BM / 2, BN);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = cluster; tile < total && ok; tile += n_clusters) {
-                const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, BM);
+                bool half;
+                const TileCoord c = decode_pair_tile(gt, p, tile, n_cols_per_tile, half);
+                const uint32_t idesc = half ? idesc_half : idesc_full;
                 const int K = c.routed ? p.K_routed : p.K_shared;
                 const int num_kb = (K + BK - 1) / BK;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, deadline)) { ok = false; break; }
@@ -172,18 +203,23 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
+        // TMEM lane l of this CTA holds, for a full tile, row 128 rank + l and all
+        // 256 columns; for a half tile (64 rows per CTA, folded), row 64 rank +
+        // (l mod 64) and columns [0,128) (l < 64) or [128,256) (l >= 64).
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
-        const int row_in_tile = static_cast<int>(rank) * BM_CTA + quarter * 32 + lane;
+        const int lane_in_cta = quarter * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = cluster; tile < total; tile += n_clusters) {
-            const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, BM);
+            bool half;
+            const TileCoord c = decode_pair_tile(gt, p, tile, n_cols_per_tile, half);
             if (!mbar_wait(&tfull[acc], acc_phase, deadline)) {
                 raise_error(p.err_flag, MOE_ERR_TIMEOUT);
                 break;
             }
             tc_fence_after();
-            const int m = c.m0 + row_in_tile;
+            const int m = c.m0 + (half ? static_cast<int>(rank) * 64 + (lane_in_cta & 63)
+                                       : static_cast<int>(rank) * BM_CTA + lane_in_cta);
             const bool valid = m < c.rows;
             const int N = c.routed ? p.N_routed : p.N_shared;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -192,11 +228,16 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(c.routed ? p.out_routed : p.out_shared);
                 const int64_t ld = c.routed ? p.ld_routed : p.ld_shared;
                 const int64_t orow = static_cast<int64_t>(gt.row0[c.g]) + m;
+                // full: gate at columns [0,128), up at [128,256) for output columns
+                // n0 + [0,128); half: gate [0,64), up [64,128) for columns
+                // n0 + 64 (l >= 64) + [0,64)
+                const int ncols = half ? 64 : BN / 2;
+                const int col0 = c.n0 + (half && lane_in_cta >= 64 ? 64 : 0);
 #pragma unroll 1
-                for (int cc = 0; cc < BN / 2; cc += 32) {
+                for (int cc = 0; cc < ncols; cc += 32) {
                     float gv[32], uv[32];
                     tmem_ld32(taddr + cc, gv);
-                    tmem_ld32(taddr + BN / 2 + cc, uv);
+                    tmem_ld32(taddr + ncols + cc, uv);
                     tmem_ld_wait();
                     uint32_t packed[16];
 #pragma unroll
@@ -207,7 +248,7 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
                         packed[j] = pack_bf16x2(h0, h1);
                     }
                     if (valid) {
-                        const int n = c.n0 + cc;
+                        const int n = col0 + cc;
                         uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + n);
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
@@ -227,8 +268,11 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
                     orow = p.out_row0_shared + gt.row0[c.g] + m;
                 }
                 const int64_t ld = p.ld_routed;
+                // full: columns n0 + [0,256); half: n0 + 128 (l >= 64) + [0,128)
+                const int ncols = half ? BN / 2 : BN;
+                const int col0 = c.n0 + (half && lane_in_cta >= 64 ? BN / 2 : 0);
 #pragma unroll 1
-                for (int cc = 0; cc < BN; cc += 32) {
+                for (int cc = 0; cc < ncols; cc += 32) {
                     float v[32];
                     tmem_ld32(taddr + cc, v);
                     tmem_ld_wait();
@@ -237,7 +281,7 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
                     for (int j = 0; j < 16; ++j)
                         packed[j] = pack_bf16x2(scale * v[2 * j], scale * v[2 * j + 1]);
                     if (valid) {
-                        const int n = c.n0 + cc;
+                        const int n = col0 + cc;
                         uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + n);
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
@@ -265,10 +309,11 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
 }
 
 static cudaError_t launch_pair(void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
-                                            GemmParams),
+                                            CUtensorMap, CUtensorMap, GemmParams),
                                int grid, cudaStream_t st, const CUtensorMap& a_r,
                                const CUtensorMap& a_s, const CUtensorMap& b_r,
-                               const CUtensorMap& b_s, const GemmParams& p) {
+                               const CUtensorMap& b_s, const CUtensorMap& bh_r,
+                               const CUtensorMap& bh_s, const GemmParams& p) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          pair::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -284,7 +329,7 @@ static cudaError_t launch_pair(void (*kern)(CUtensorMap, CUtensorMap, CUtensorMa
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a_r, a_s, b_r, b_s, p);
+    return cudaLaunchKernelEx(&cfg, kern, a_r, a_s, b_r, b_s, bh_r, bh_s, p);
 }
 
 // GEMM 1 (gate_up + SwiGLU) and GEMM 2 (down + weight) on CTA pairs.
@@ -299,19 +344,21 @@ cudaError_t launch_ffn_sm100_pair(const moe_shape& s, const void* x, const void*
     const int S = s.n_shared;
     const int Is = S > 0 ? s.I_shared : s.I;
 
-    CUtensorMap a1r, a1s, b1r, b1s, a2r, a2s, b2r, b2s;
+    CUtensorMap a1r, a1s, b1r, b1s, h1r, h1s, a2r, a2s, b2r, b2s;
     bool ok = true;
     ok &= make_map(&a1r, x_perm, Tk, s.H, BM_CTA);
     ok &= make_map(&b1r, gate_up, static_cast<int64_t>(s.E) * 2 * s.I, s.H, BN_CTA);
+    ok &= make_map(&h1r, gate_up, static_cast<int64_t>(s.E) * 2 * s.I, s.H, BN_CTA / 2);
     ok &= make_map(&a2r, h_routed, Tk, s.I, BM_CTA);
     ok &= make_map(&b2r, down, static_cast<int64_t>(s.E) * s.H, s.I, BN_CTA);
     if (S > 0) {
         ok &= make_map(&a1s, x, s.T, s.H, BM_CTA);
         ok &= make_map(&b1s, sh_gate_up, static_cast<int64_t>(S) * 2 * Is, s.H, BN_CTA);
+        ok &= make_map(&h1s, sh_gate_up, static_cast<int64_t>(S) * 2 * Is, s.H, BN_CTA / 2);
         ok &= make_map(&a2s, h_shared, static_cast<int64_t>(S) * s.T, Is, BM_CTA);
         ok &= make_map(&b2s, sh_down, static_cast<int64_t>(S) * s.H, Is, BN_CTA);
     } else {
-        a1s = a1r; b1s = b1r; a2s = a2r; b2s = b2r;
+        a1s = a1r; b1s = b1r; h1s = h1r; a2s = a2r; b2s = b2r;
     }
     if (!ok) return cudaErrorInvalidValue;
 
@@ -350,7 +397,8 @@ cudaError_t launch_ffn_sm100_pair(const moe_shape& s, const void* x, const void*
     p.out_row0_shared = 0;
     int64_t tiles = mt_bound * p.n_tiles_routed + mt_shared * p.n_tiles_shared;
     int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
-    cudaError_t e = launch_pair(grouped_gemm_pair<kSwiGLU>, 2 * clusters, st, a1r, a1s, b1r, b1s, p);
+    cudaError_t e = launch_pair(grouped_gemm_pair<kSwiGLU>, 2 * clusters, st, a1r, a1s, b1r, b1s,
+                                h1r, h1s, p);
     if (e != cudaSuccess) return e;
 
     // GEMM 2
@@ -371,7 +419,8 @@ cudaError_t launch_ffn_sm100_pair(const moe_shape& s, const void* x, const void*
     p.out_row0_shared = Tk;
     tiles = mt_bound * p.n_tiles_routed + mt_shared * p.n_tiles_shared;
     clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
-    return launch_pair(grouped_gemm_pair<kScaled>, 2 * clusters, st, a2r, a2s, b2r, b2s, p);
+    return launch_pair(grouped_gemm_pair<kScaled>, 2 * clusters, st, a2r, a2s, b2r, b2s, b2r, b2s,
+                       p);
 }
 
 }  // namespace moe

@@ -188,13 +188,19 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* off
     void* x_perm = ws + w.x_perm_off;
     cudaError_t e = moe::launch_gather_rows(s, x, perm, x_perm, sms, cs);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-#ifndef MOE_GEMM_PAIR
-#define MOE_GEMM_PAIR 1
+    // CTA pairs (256-row tiles) when the experts average at least 256 rows;
+    // one CTA per tile otherwise (less padding on small groups)
+#ifndef MOE_PAIR_MIN_ROWS
+#define MOE_PAIR_MIN_ROWS 256
 #endif
-    if (MOE_GEMM_PAIR)
+#ifndef MOE_PAIR_GROUP_M
+#define MOE_PAIR_GROUP_M 16
+#endif
+    if (s.T * s.k >= static_cast<int64_t>(MOE_PAIR_MIN_ROWS) * s.E)
         return cuda_status(moe::launch_ffn_sm100_pair(s, x, x_perm, offsets, perm, topk_w, gate_up,
                                                       down, sh_gate_up, sh_down, h_routed,
-                                                      h_shared, y_slots, err_flag, sms, 4, cs));
+                                                      h_shared, y_slots, err_flag, sms,
+                                                      MOE_PAIR_GROUP_M, cs));
     return cuda_status(moe::launch_ffn_sm100(s, x, x_perm, offsets, perm, topk_w, gate_up, down,
                                              sh_gate_up, sh_down, h_routed, h_shared, y_slots,
                                              err_flag, sms, 8, cs));

@@ -34,6 +34,12 @@ SMALL = [
               routed_scale=2.5),
     MoEConfig("bf16_decode_T8", T=8, H=1024, I=512, E=4, k=4),
     MoEConfig("bf16_just_above_decode", T=9, H=256, I=256, E=8, k=2),
+    # >= 256 rows per expert on average: CTA-pair kernel, incl. 64-row-per-CTA
+    # half tiles for group tails of <= 128 rows, ragged N and K, shared experts
+    MoEConfig("pair_ragged", T=1100, H=712, I=328, E=4, k=2),
+    MoEConfig("pair_shared_zipf", T=600, H=256, I=256, E=4, k=2, n_shared=2, I_shared=136,
+              routed_scale=2.5, zipf_s=1.0),
+    MoEConfig("pair_many_groups", T=1536, H=384, I=200, E=12, k=3, zipf_s=1.2),
 ]
 
 
