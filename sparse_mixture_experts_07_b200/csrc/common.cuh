@@ -51,13 +51,15 @@ template <> struct ElemIO<__nv_bfloat16> {
 // rows are [offsets[g], offsets[g+1]) of the sorted slot space; group E + s is
 // shared expert s whose rows are the T tokens.  The table is rebuilt by every
 // CTA from the device offsets, so the host never reads the expert counts.
-struct GroupTable {
+template <int MAXG>
+struct GroupTableT {
     int32_t n_groups;
     int32_t total_tiles;
-    int32_t tile_start[kMaxGroups + 1];   // prefix over groups of tiles
-    int32_t rows[kMaxGroups];             // M of each group
-    int32_t row0[kMaxGroups];             // first row of the group in its A space
+    int32_t tile_start[MAXG + 1];   // prefix over groups of tiles
+    int32_t rows[MAXG];             // M of each group
+    int32_t row0[MAXG];             // first row of the group in its A space
 };
+using GroupTable = GroupTableT<kMaxGroups>;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers (sm_100a).
@@ -286,7 +288,8 @@ namespace moe {
 // Builds the group table (one thread; at most kMaxGroups iterations).
 // Routed group g covers rows [offsets[g], offsets[g+1]); shared group E+s
 // covers the T token rows.  Tiles of a group: ceil(rows / BM) * n_tiles.
-__device__ __forceinline__ void build_group_table(GroupTable& gt, const int32_t* offsets, int E,
+template <int MAXG>
+__device__ __forceinline__ void build_group_table(GroupTableT<MAXG>& gt, const int32_t* offsets, int E,
                                                   int S, int64_t T, int BM, int n_tiles_routed,
                                                   int n_tiles_shared) {
     int32_t acc = 0;
@@ -313,7 +316,8 @@ __device__ __forceinline__ void build_group_table(GroupTable& gt, const int32_t*
 }
 
 // Group of a linear tile index (binary search over the prefix).
-__device__ __forceinline__ int find_group(const GroupTable& gt, int32_t tile) {
+template <int MAXG>
+__device__ __forceinline__ int find_group(const GroupTableT<MAXG>& gt, int32_t tile) {
     int lo = 0, hi = gt.n_groups - 1;
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;

@@ -37,7 +37,8 @@ struct TileCoord {
     bool routed;
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const GroupTable& gt, const GemmParams& p,
+template <int MAXG>
+__device__ __forceinline__ TileCoord decode_tile(const GroupTableT<MAXG>& gt, const GemmParams& p,
                                                  int tile, int n_cols_per_tile, int BM) {
     TileCoord c;
     c.g = find_group(gt, tile);

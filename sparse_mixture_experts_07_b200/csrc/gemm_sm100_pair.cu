@@ -32,28 +32,31 @@ constexpr int BN = 256;                       // MMA N
 constexpr int BN_CTA = 128;                   // B rows per CTA
 constexpr int BK = 64;
 constexpr int UMMA_K = 16;
-constexpr int STAGES = 6;
 constexpr int A_BYTES = BM_CTA * BK * 2;      // 16 KB
 constexpr int B_BYTES = BN_CTA * BK * 2;      // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 512;                // two 256-column accumulators
 constexpr int THREADS = 192;
 constexpr int EPI_WARPS = 4;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint16_t BOTH = 0x3;                // cluster ranks 0 and 1
 }  // namespace pair
+
+constexpr int kSmallGroups = 72;              // E + S of every shape measured here
 
 // Tile of the pair kernel.  The last m-tile of a group is a "half" tile when
 // at most 128 of its rows are real: it runs as an M=128 pair MMA (64 rows per
 // CTA) instead of M=256, which halves the padding of that tile.
-__device__ __forceinline__ TileCoord decode_pair_tile(const GroupTable& gt, const GemmParams& p,
+template <int MAXG>
+__device__ __forceinline__ TileCoord decode_pair_tile(const GroupTableT<MAXG>& gt, const GemmParams& p,
                                                       int tile, int n_cols_per_tile, bool& half) {
     const TileCoord c = decode_tile(gt, p, tile, n_cols_per_tile, pair::BM);
     half = c.rows - c.m0 <= pair::BM / 2;
     return c;
 }
 
-template <int EPI>
+// STAGES: depth of the shared-memory ring (7 fits next to a group table of at
+// most 72 groups, 6 next to the full 264).
+template <int EPI, int STAGES, int MAXG>
 __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
     const __grid_constant__ CUtensorMap map_a_routed, const __grid_constant__ CUtensorMap map_a_shared,
     const __grid_constant__ CUtensorMap map_b_routed, const __grid_constant__ CUtensorMap map_b_shared,
@@ -61,7 +64,7 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
     const __grid_constant__ CUtensorMap map_bh_shared, const GemmParams p) {
     using namespace pair;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ GroupTable gt;
+    __shared__ GroupTableT<MAXG> gt;
     __shared__ uint32_t tmem_base_sh;
 
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -308,19 +311,21 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
     }
 }
 
+constexpr int pair_smem_bytes(int stages) { return stages * pair::STAGE_BYTES + 1024 + 256; }
+
 static cudaError_t launch_pair(void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
                                             CUtensorMap, CUtensorMap, GemmParams),
-                               int grid, cudaStream_t st, const CUtensorMap& a_r,
+                               int smem_bytes, int grid, cudaStream_t st, const CUtensorMap& a_r,
                                const CUtensorMap& a_s, const CUtensorMap& b_r,
                                const CUtensorMap& b_s, const CUtensorMap& bh_r,
                                const CUtensorMap& bh_s, const GemmParams& p) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         pair::SMEM_BYTES);
+                                         smem_bytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.blockDim = dim3(pair::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -397,8 +402,14 @@ cudaError_t launch_ffn_sm100_pair(const moe_shape& s, const void* x, const void*
     p.out_row0_shared = 0;
     int64_t tiles = mt_bound * p.n_tiles_routed + mt_shared * p.n_tiles_shared;
     int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
-    cudaError_t e = launch_pair(grouped_gemm_pair<kSwiGLU>, 2 * clusters, st, a1r, a1s, b1r, b1s,
-                                h1r, h1s, p);
+    // a deeper ring when the group table is small enough to leave room for it
+    const bool deep = s.E + S <= kSmallGroups;
+    cudaError_t e = deep ? launch_pair(grouped_gemm_pair<kSwiGLU, 7, kSmallGroups>,
+                                       pair_smem_bytes(7), 2 * clusters, st, a1r, a1s, b1r, b1s,
+                                       h1r, h1s, p)
+                         : launch_pair(grouped_gemm_pair<kSwiGLU, 6, kMaxGroups>,
+                                       pair_smem_bytes(6), 2 * clusters, st, a1r, a1s, b1r, b1s,
+                                       h1r, h1s, p);
     if (e != cudaSuccess) return e;
 
     // GEMM 2
@@ -419,8 +430,10 @@ cudaError_t launch_ffn_sm100_pair(const moe_shape& s, const void* x, const void*
     p.out_row0_shared = Tk;
     tiles = mt_bound * p.n_tiles_routed + mt_shared * p.n_tiles_shared;
     clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
-    return launch_pair(grouped_gemm_pair<kScaled>, 2 * clusters, st, a2r, a2s, b2r, b2s, b2r, b2s,
-                       p);
+    return deep ? launch_pair(grouped_gemm_pair<kScaled, 7, kSmallGroups>, pair_smem_bytes(7),
+                              2 * clusters, st, a2r, a2s, b2r, b2s, b2r, b2s, p)
+                : launch_pair(grouped_gemm_pair<kScaled, 6, kMaxGroups>, pair_smem_bytes(6),
+                              2 * clusters, st, a2r, a2s, b2r, b2s, b2r, b2s, p);
 }
 
 }  // namespace moe
