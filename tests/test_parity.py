@@ -146,3 +146,27 @@ def test_bounded_wait_expires_and_reports_timeout(cuda_ok):
     inp, res = _run(cfg)
     assert res["err"] == 0
     check_routing(cfg, inp, res)
+
+
+def test_token_permutation_permutes_output_rows_exactly(cuda_ok):
+    """Each output row depends only on its own token: permuting the tokens
+    permutes the rows of y bit for bit (pair kernel, half tiles included)."""
+    cfg = MoEConfig("perm_inv", T=1200, H=256, I=192, E=4, k=2, n_shared=1, I_shared=64,
+                    routed_scale=2.5)
+    inp = make_inputs(cfg)
+    a = run_gpu(cfg, to_device(inp))
+    pi = torch.from_numpy(np.random.default_rng(0).permutation(cfg.T))
+    inp2 = dict(inp)
+    inp2["x"] = inp["x"][pi]
+    b = run_gpu(cfg, to_device(inp2))
+    assert torch.equal(b["topk_idx"], a["topk_idx"][pi])
+    assert torch.equal(b["y"], a["y"][pi])
+
+
+def test_pair_kernel_repeat_runs_are_bit_identical(cuda_ok):
+    cfg = MoEConfig("det_pair", T=2048, H=512, I=384, E=8, k=2, zipf_s=1.0)
+    inp = to_device(make_inputs(cfg))
+    a = run_gpu(cfg, inp)
+    b = run_gpu(cfg, inp)
+    for key in ("topk_idx", "perm", "y_slots", "y"):
+        assert torch.equal(a[key], b[key])
