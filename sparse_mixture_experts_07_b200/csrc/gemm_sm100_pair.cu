@@ -119,6 +119,13 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
+#ifndef MOE_PAIR_L2_HINTS
+#define MOE_PAIR_L2_HINTS 1
+#endif
+            // L2 priorities: activation rows are reused by every n-tile of their
+            // group, weight panels only by the few m-tiles of one band
+            const uint64_t pol_a = MOE_PAIR_L2_HINTS ? l2_policy_evict_last() : l2_policy_evict_normal();
+            const uint64_t pol_b = MOE_PAIR_L2_HINTS >= 2 ? l2_policy_evict_first() : l2_policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -150,12 +157,13 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const uint32_t bar = full_leader + stage * 8;
-                    tma_load_2d_pair(sa, ma, bar, kb * BK, a_row);
+                    tma_load_2d_pair_hint(sa, ma, bar, kb * BK, a_row, pol_a);
                     if (EPI == kSwiGLU && half) {
-                        tma_load_2d_pair(sa + A_BYTES, mbh, bar, kb * BK, b_row);
-                        tma_load_2d_pair(sa + A_BYTES + B_BYTES / 2, mbh, bar, kb * BK, b_row + up_off);
+                        tma_load_2d_pair_hint(sa + A_BYTES, mbh, bar, kb * BK, b_row, pol_b);
+                        tma_load_2d_pair_hint(sa + A_BYTES + B_BYTES / 2, mbh, bar, kb * BK,
+                                              b_row + up_off, pol_b);
                     } else {
-                        tma_load_2d_pair(sa + A_BYTES, mb, bar, kb * BK, b_row);
+                        tma_load_2d_pair_hint(sa + A_BYTES, mb, bar, kb * BK, b_row, pol_b);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
