@@ -38,8 +38,8 @@ L2_BYTES = 126 * 1024 * 1024
 # kernels, from one ncu capture, keyed by workload; valid only while the GEMM
 # source is unchanged (sha256 of the file, first 16 hex digits).
 TRAFFIC = {
-    # profiles/grouped_gemm_pair_mixtral.md: gather 0.054 + GEMM 1 3.723 + GEMM 2 1.905 GB
-    "mixtral": {"bytes": 5.682e9, "file": "gemm_sm100_pair.cu", "sha": "c248fc56b2007956"},
+    # profiles/grouped_gemm_pair_mixtral.md: gather 0.054 + GEMM 1 2.385 + GEMM 2 1.484 GB
+    "mixtral": {"bytes": 3.923e9, "file": "gemm_sm100_pair.cu", "sha": "dd8fdb2089d58863"},
 }
 
 
