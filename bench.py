@@ -260,6 +260,7 @@ def run_cuda(args, cfg, rank, local, world):
         s0.record(stream)
         for i in range(args.steps):
             idx, w, _ = moe.route(shape, x, layer.w_router, layer.router_bias, out=b,
+                                  w_split=layer.w_split,
                                   err_flag=layer.err_flag)
             moe.permute(shape, idx, layer.workspace, layer.err_flag, out=b)
             fwd_start[i].record(stream)

@@ -115,6 +115,42 @@ MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const float*
                              const float* router_bias, float* logits, int32_t* topk_idx,
                              float* topk_w, int32_t* err_flag, void* stream);
 
+/* The float32 router weight split into three bf16 terms ahead of time, for the
+ * tensor-core router.  The split depends on the weight alone, so a caller does
+ * it once when the weights are loaded ("Mixture of Experts in Transformers",
+ * WeightConverter section: conversions belong to the weight-loading
+ * pipeline), not on every call.
+ *
+ * moe_router_split_size writes to *bytes the size of the split weight for
+ * `shape`: N * H * 2 bytes with E_PAD = 8, 16, 32 or 64 (the smallest >= E) and
+ * N = 3 * E_PAD rounded up to a multiple of 16; 0 when the tensor-core router
+ * does not apply (float32 x, or E > 64).
+ *
+ * moe_router_split fills
+ *   w_split  [N, H]  bf16 output, 16-byte aligned, caller-owned: row e is
+ *                    hi(W[e]), row E_PAD + e is mid(W[e]), row 2 E_PAD + e is
+ *                    lo(W[e]) where hi = bf16(w), mid = bf16(w - hi),
+ *                    lo = bf16(w - hi - mid) (round to nearest even), so
+ *                    hi + mid + lo equals w to within 2^-24 |w|; rows of
+ *                    experts >= E and rows >= 3 E_PAD are zero.
+ * It returns MOE_ERR_UNSUPPORTED when the size above is 0 or a pointer is not
+ * 16-byte aligned, and MOE_ERR_WORKSPACE when w_split_bytes is too small.
+ *
+ * moe_route_split computes exactly what moe_route computes, with the same
+ * arguments plus `w_split` (the output of moe_router_split for this shape and
+ * weight, or NULL).  For more than 256 tokens with bf16 x and E <= 64 it runs
+ * the tensor-core router on w_split; its results are bit-identical to
+ * moe_route's.  Otherwise, or when w_split is NULL, it is moe_route.
+ * A w_split that does not match w_router gives the routing of the weight it
+ * was split from. */
+MOE_API moe_status moe_router_split_size(const moe_shape* shape, size_t* bytes);
+MOE_API moe_status moe_router_split(const moe_shape* shape, const float* w_router, void* w_split,
+                                    size_t w_split_bytes, void* stream);
+MOE_API moe_status moe_route_split(const moe_shape* shape, const void* x, const float* w_router,
+                                   const void* w_split, const float* router_bias, float* logits,
+                                   int32_t* topk_idx, float* topk_w, int32_t* err_flag,
+                                   void* stream);
+
 /* Dropless dispatch plan ("Mixture of Experts in Transformers", grouped_mm
  * backend: sort and group tokens by expert id).  Slot q = t*k + j.
  *   topk_idx  [T, k]  int32 input

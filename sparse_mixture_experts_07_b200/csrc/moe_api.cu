@@ -9,6 +9,10 @@ cudaError_t launch_route(const moe_shape&, const void*, const float*, const floa
                          int32_t*, float*, cudaStream_t);
 cudaError_t launch_route_tc(const moe_shape&, const void*, const float*, const float*, float*,
                             int32_t*, float*, int32_t*, cudaStream_t);
+int router_split_rows(const moe_shape&);
+cudaError_t launch_router_split(const moe_shape&, const float*, void*, int, cudaStream_t);
+cudaError_t launch_route_tc_split(const moe_shape&, const void*, const void*, const float*, float*,
+                                  int32_t*, float*, int32_t*, int, cudaStream_t);
 cudaError_t launch_route_small(const moe_shape&, const void*, const float*, const float*, float*,
                                int32_t*, float*, cudaStream_t);
 size_t permute_workspace_bytes(const moe_shape&);
@@ -135,6 +139,45 @@ moe_status moe_route(const moe_shape* shape, const void* x, const float* w_route
                                                 topk_idx, topk_w, err_flag, cs));
     return cuda_status(moe::launch_route(*shape, x, w_router, router_bias, logits, topk_idx,
                                          topk_w, cs));
+}
+
+moe_status moe_router_split_size(const moe_shape* shape, size_t* bytes) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = static_cast<size_t>(moe::router_split_rows(*shape)) * shape->H * 2;
+    return MOE_OK;
+}
+
+moe_status moe_router_split(const moe_shape* shape, const float* w_router, void* w_split,
+                            size_t w_split_bytes, void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    const size_t need = static_cast<size_t>(moe::router_split_rows(*shape)) * shape->H * 2;
+    if (need == 0) return MOE_ERR_UNSUPPORTED;
+    if (!w_router || !w_split) return MOE_ERR_INVALID_ARG;
+    if (w_split_bytes < need) return MOE_ERR_WORKSPACE;
+    if (!aligned16(w_router) || !aligned16(w_split)) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(moe::launch_router_split(*shape, w_router, w_split, num_sms(),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_route_split(const moe_shape* shape, const void* x, const float* w_router,
+                           const void* w_split, const float* router_bias, float* logits,
+                           int32_t* topk_idx, float* topk_w, int32_t* err_flag, void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    // the split weight serves the tensor-core path; everything else is moe_route
+    const bool tc = shape->T > 256 && moe::router_split_rows(*shape) > 0;
+    if (!tc || !w_split)
+        return moe_route(shape, x, w_router, router_bias, logits, topk_idx, topk_w, err_flag,
+                         stream);
+    if (!aligned16(x) || !aligned16(w_split)) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(moe::launch_route_tc_split(*shape, x, w_split, router_bias, logits,
+                                                  topk_idx, topk_w, err_flag, num_sms(),
+                                                  static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,

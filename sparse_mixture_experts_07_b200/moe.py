@@ -20,7 +20,7 @@ MOE_F32, MOE_BF16 = 0, 1
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_INDEX", 6: "MOE_ERR_TIMEOUT"}
 EXPORTS = ("moe_status_str", "moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
-           "moe_combine")
+           "moe_combine", "moe_router_split_size", "moe_router_split", "moe_route_split")
 
 
 class MoEShape(ctypes.Structure):
@@ -57,6 +57,9 @@ def load_library(path: str = LIB_PATH):
     lib.moe_permute.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_combine.argtypes = [S, P, P, P, P]
+    lib.moe_router_split_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
+    lib.moe_router_split.argtypes = [S, P, P, ctypes.c_size_t, P]
+    lib.moe_route_split.argtypes = [S, P, P, P, P, P, P, P, P, P]
     for f in EXPORTS[1:]:
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -118,17 +121,40 @@ def alloc_workspace(shape: Shape, device="cuda") -> torch.Tensor:
     return torch.empty(max(workspace_size(shape), 1), dtype=torch.uint8, device=device)
 
 
+def router_split(shape: Shape, w_router, stream=None):
+    """The router weight split into three bf16 terms [N, H] (hi, mid, lo planes of
+    E_PAD rows each, zero padding), for the tensor-core router; None when that
+    router does not apply to `shape`.  Done once per weight."""
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    _check(lib.moe_router_split_size(ctypes.byref(shape.c()), ctypes.byref(n)),
+           "moe_router_split_size")
+    if n.value == 0:
+        return None
+    ws = torch.empty(n.value // (2 * shape.H), shape.H, dtype=torch.bfloat16,
+                     device=w_router.device)
+    _check(lib.moe_router_split(ctypes.byref(shape.c()), _ptr(w_router), _ptr(ws), n.value,
+                                _stream(stream)), "moe_router_split")
+    return ws
+
+
 def route(shape: Shape, x, w_router, router_bias=None, logits=False, out=None, stream=None,
-          err_flag=None):
-    """(topk_idx [T,k] int32, topk_w [T,k] f32, logits [T,E] f32 or None)."""
+          err_flag=None, w_split=None):
+    """(topk_idx [T,k] int32, topk_w [T,k] f32, logits [T,E] f32 or None).
+    `w_split` (from router_split) lets large batches skip the weight split."""
     lib = load_library()
     dev = x.device
     idx = out["topk_idx"] if out else torch.empty(shape.T, shape.k, dtype=torch.int32, device=dev)
     w = out["topk_w"] if out else torch.empty(shape.T, shape.k, dtype=torch.float32, device=dev)
     lg = torch.empty(shape.T, shape.E, dtype=torch.float32, device=dev) if logits else None
-    _check(lib.moe_route(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(router_bias),
-                         _ptr(lg), _ptr(idx), _ptr(w), _ptr(err_flag), _stream(stream)),
-           "moe_route")
+    if w_split is not None:
+        _check(lib.moe_route_split(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router),
+                                   _ptr(w_split), _ptr(router_bias), _ptr(lg), _ptr(idx), _ptr(w),
+                                   _ptr(err_flag), _stream(stream)), "moe_route_split")
+    else:
+        _check(lib.moe_route(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(router_bias),
+                             _ptr(lg), _ptr(idx), _ptr(w), _ptr(err_flag), _stream(stream)),
+               "moe_route")
     return idx, w, lg
 
 
@@ -186,6 +212,8 @@ class MoELayer:
                  sh_down=None):
         self.shape = shape
         self.w_router, self.router_bias = w_router, router_bias
+        # split once here, at load time; refresh it if w_router changes
+        self.w_split = router_split(shape, w_router)
         self.gate_up, self.down = gate_up, down
         self.sh_gate_up, self.sh_down = sh_gate_up, sh_down
         dev = gate_up.device
@@ -207,7 +235,7 @@ class MoELayer:
     def __call__(self, x, stream=None, y=None):
         s, b = self.shape, self.buf
         idx, w, _ = route(s, x, self.w_router, self.router_bias, out=b, stream=stream,
-                          err_flag=self.err_flag)
+                          err_flag=self.err_flag, w_split=self.w_split)
         counts, offsets, perm, inv = permute(s, idx, self.workspace, self.err_flag, out=b,
                                              stream=stream)
         forward(s, x, offsets, perm, w, self.gate_up, self.down, self.sh_gate_up, self.sh_down,

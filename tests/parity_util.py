@@ -39,8 +39,12 @@ def run_gpu(cfg: MoEConfig, dinp: dict) -> dict:
     shape = moe.Shape.from_config(cfg)
     layer = moe.MoELayer(shape, dinp["w_router"], dinp["router_bias"], dinp["gate_up"],
                          dinp["down"], dinp["sh_gate_up"], dinp["sh_down"])
+    # logits of the router that splits the weight in every CTA, and of the
+    # router on the weight split at load time (the layer's path)
     idx, w, logits = moe.route(shape, dinp["x"], dinp["w_router"], dinp["router_bias"],
                                logits=True)
+    _, _, logits_split = moe.route(shape, dinp["x"], dinp["w_router"], dinp["router_bias"],
+                                   logits=True, w_split=layer.w_split)
     y = layer(dinp["x"])
     torch.cuda.synchronize()
     b = layer.last
@@ -48,6 +52,7 @@ def run_gpu(cfg: MoEConfig, dinp: dict) -> dict:
                                          "y_slots")}
     res["y"] = y.cpu()
     res["logits"] = logits.cpu()
+    res["logits_split"] = logits_split.cpu()
     res["route_idx"] = idx.cpu()
     res["err"] = layer.device_error()
     return res
@@ -71,6 +76,8 @@ def check_routing(cfg: MoEConfig, inp: dict, res: dict, tokens=None):
     sel = slice(None) if tokens is None else np.asarray(tokens)
     assert np.array_equal(g_idx[sel], o_idx), "routing indices differ"
     lerr = float(np.abs(res["logits"].numpy()[sel] - lg).max())
+    if "logits_split" in res:
+        lerr = max(lerr, float(np.abs(res["logits_split"].numpy()[sel] - lg).max()))
     werr = float(np.abs(g_w[sel] - o_w).max())
     ltol = logit_tol(cfg.H, lg)
     assert lerr <= ltol, f"logit error {lerr:.3e} > {ltol:.3e}"

@@ -112,6 +112,46 @@ def test_misaligned_bf16_pointers_rejected(lib):
     assert lib.moe_combine(ctypes.byref(s), bad, ok, ok, None) == 2
 
 
+def _split_size(lib, s):
+    n = ctypes.c_size_t(0)
+    rc = lib.moe_router_split_size(ctypes.byref(s), ctypes.byref(n))
+    return rc, n.value
+
+
+@pytest.mark.parametrize("E,rows", [(1, 32), (8, 32), (9, 48), (16, 48), (17, 96), (32, 96), (40, 192),
+                                    (64, 192)])
+def test_router_split_size(lib, E, rows):
+    # N = 3 E_PAD rounded up to 16, E_PAD in {8, 16, 32, 64}; bf16 rows of H
+    assert _split_size(lib, _shape(E=E, k=1, H=256)) == (0, rows * 256 * 2)
+
+
+def test_router_split_size_zero_where_the_tensor_core_router_does_not_apply(lib):
+    assert _split_size(lib, _shape(dtype=moe.MOE_F32)) == (0, 0)
+    assert _split_size(lib, _shape(E=65)) == (0, 0)
+    assert _split_size(lib, _shape(k=0))[0] == 1
+
+
+def test_router_split_argument_checks(lib):
+    s = _shape(E=8, H=128)
+    _, need = _split_size(lib, s)
+    ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 4)
+    assert lib.moe_router_split(ctypes.byref(s), None, ok, need, None) == 1
+    assert lib.moe_router_split(ctypes.byref(s), ok, None, need, None) == 1
+    assert lib.moe_router_split(ctypes.byref(s), ok, ok, need - 1, None) == 3
+    assert lib.moe_router_split(ctypes.byref(s), bad, ok, need, None) == 2
+    assert lib.moe_router_split(ctypes.byref(s), ok, bad, need, None) == 2
+    f32 = _shape(dtype=moe.MOE_F32)
+    assert lib.moe_router_split(ctypes.byref(f32), ok, ok, 1 << 20, None) == 2
+    p = ctypes.c_void_p(16)
+    assert lib.moe_route_split(ctypes.byref(s), None, p, p, None, None, p, p, None, None) == 1
+    assert lib.moe_route_split(ctypes.byref(s), p, None, p, None, None, p, p, None, None) == 1
+    big = _shape(T=4096, E=8)
+    assert lib.moe_route_split(ctypes.byref(big), bad, ok, ok, None, None, ok, ok, None,
+                               None) == 2
+    assert lib.moe_route_split(ctypes.byref(big), ok, ok, bad, None, None, ok, ok, None,
+                               None) == 2
+
+
 def test_zero_tokens_is_a_no_op(lib):
     s = _shape(T=0)
     assert lib.moe_route(ctypes.byref(s), None, None, None, None, None, None, None, None) == 0

@@ -170,3 +170,54 @@ def test_pair_kernel_repeat_runs_are_bit_identical(cuda_ok):
     b = run_gpu(cfg, inp)
     for key in ("topk_idx", "perm", "y_slots", "y"):
         assert torch.equal(a[key], b[key])
+
+
+@pytest.mark.parametrize("E,H", [(8, 4096), (40, 200), (64, 2048)])
+def test_router_split_planes_sum_to_the_weight(cuda_ok, E, H):
+    """hi + mid + lo equals each float32 router weight to within 2^-24 |w|;
+    padding rows (experts >= E, rows >= 3 E_PAD) are zero."""
+    import sparse_mixture_experts_07_b200 as moe
+    shape = moe.Shape(T=512, H=H, I=128, E=E, k=2)
+    g = torch.Generator().manual_seed(E)
+    w = (torch.randn(E, H, generator=g) * 0.02).cuda()
+    ws = moe.router_split(shape, w)
+    torch.cuda.synchronize()
+    e_pad = next(p for p in (8, 16, 32, 64) if p >= E)
+    assert ws.shape == ((3 * e_pad + 15) // 16 * 16, H)
+    planes = ws.double().cpu()
+    total = planes[:E] + planes[e_pad:e_pad + E] + planes[2 * e_pad:2 * e_pad + E]
+    wd = w.double().cpu()
+    assert torch.all((total - wd).abs() <= 2.0 ** -24 * wd.abs())
+    pad = torch.ones(planes.shape[0], dtype=torch.bool)
+    for t in range(3):
+        pad[t * e_pad:t * e_pad + E] = False
+    assert torch.all(planes[pad] == 0)
+
+
+@pytest.mark.parametrize("cfg", [
+    MoEConfig("split_E8", T=1000, H=512, I=64, E=8, k=2),
+    MoEConfig("split_E40_ragged_H", T=700, H=200, I=64, E=40, k=3, zipf_s=1.0),
+    MoEConfig("split_E64", T=2100, H=256, I=64, E=64, k=6, zipf_s=1.2),
+    MoEConfig("split_k8_E16", T=300, H=4096, I=64, E=16, k=2),
+    MoEConfig("split_k4_E64_ragged", T=1000, H=2056, I=64, E=64, k=6, zipf_s=1.2),
+], ids=lambda c: c.name)
+def test_route_with_presplit_weight_matches_route(cuda_ok, cfg):
+    """The router on the weight split at load time (split-K over a cluster
+    when the m-tiles leave SMs idle) selects exactly what the router that
+    splits the weight in every CTA selects; logits and weights agree within
+    the float32 summation bound; repeated calls are bit-identical."""
+    import sparse_mixture_experts_07_b200 as moe
+    from parity_util import logit_tol
+    inp = to_device(make_inputs(cfg))
+    shape = moe.Shape.from_config(cfg)
+    ws = moe.router_split(shape, inp["w_router"])
+    a = moe.route(shape, inp["x"], inp["w_router"], inp["router_bias"], logits=True)
+    b = moe.route(shape, inp["x"], inp["w_router"], inp["router_bias"], logits=True, w_split=ws)
+    c = moe.route(shape, inp["x"], inp["w_router"], inp["router_bias"], logits=True, w_split=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0])
+    tol = logit_tol(cfg.H, a[2].cpu().numpy())
+    assert float((a[2] - b[2]).abs().max()) <= tol
+    assert float((a[1] - b[1]).abs().max()) <= 2 * tol
+    for u, v in zip(b, c):
+        assert torch.equal(u, v)
