@@ -14,8 +14,13 @@
 //   3. scatter: each block ranks its slots stably (warp match + per-warp
 //      counts, rounds in slot order) and writes perm and inv.
 // The order (expert ascending, slot ascending) is fixed, so the plan is
-// bit-identical run to run.  Workspace: nblocks * E int32.  A plan of a
-// single block (T*k <= 2048) runs all three steps in one CTA and one launch.
+// bit-identical run to run.  Workspace: nblocks * E int32.
+//
+// Up to 8 * 8 * 1024 slots, the plan runs instead as ONE launch on one
+// thread-block cluster of up to 8 CTAs of 1024 threads (permute_cluster_kernel):
+// each CTA counts its contiguous slice of slots, reads the other CTAs'
+// counts from their shared memory (DSMEM) to find its starting position per
+// expert, and ranks its slots with the same stable scheme.  No workspace.
 #include "common.cuh"
 
 namespace moe {
@@ -85,69 +90,115 @@ __global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(
 __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
     const int32_t* __restrict__ idx, int64_t n, int E, const int32_t* __restrict__ blk_base,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
-    __shared__ int32_t running[kMaxExperts];
+    __shared__ int32_t running[2][kMaxExperts];
+    // per-warp counts of the current round, stamped with the round in the high
+    // half so that entries left from earlier rounds read as zero
     __shared__ int32_t wcnt[kPermThreads / 32][kMaxExperts];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int e = tid; e < E; e += kPermThreads)
-        running[e] = blk_base[static_cast<int64_t>(blockIdx.x) * E + e];
+        running[0][e] = blk_base[static_cast<int64_t>(blockIdx.x) * E + e];
+    for (int i = tid; i < (kPermThreads / 32) * kMaxExperts; i += kPermThreads)
+        (&wcnt[0][0])[i] = -1;
     const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermSlotsPerBlock;
+    int ev[kPermRounds];
+#pragma unroll
     for (int r = 0; r < kPermRounds; ++r) {
-        for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads)
-            wcnt[i / E][i % E] = 0;
-        __syncthreads();
         const int64_t q = base + r * kPermThreads + tid;
-        int e = -1;
-        if (q < n) {
-            e = idx[q];
-            if (e < 0 || e >= E) e = -1;
-        }
+        int e = q < n ? idx[q] : -1;
+        ev[r] = (e >= 0 && e < E) ? e : -1;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kPermRounds; ++r) {
+        const int cur = r & 1;
+        const int e = ev[r];
+        const int64_t q = base + r * kPermThreads + tid;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int lane_rank = __popc(peers & ((1u << lane) - 1u));
-        if (e >= 0 && lane_rank == 0) wcnt[warp][e] = __popc(peers);
+        if (e >= 0 && lane_rank == 0) wcnt[warp][e] = (r << 16) | __popc(peers);
         __syncthreads();
         if (e >= 0) {
-            int32_t p = running[e] + lane_rank;
-            for (int w = 0; w < warp; ++w) p += wcnt[w][e];
+            int32_t p = running[cur][e] + lane_rank;
+            for (int w = 0; w < warp; ++w) {
+                const int32_t v = wcnt[w][e];
+                if ((v >> 16) == r) p += v & 0xffff;
+            }
             perm[p] = static_cast<int32_t>(q);
             inv[q] = p;
         }
-        __syncthreads();
         for (int ee = tid; ee < E; ee += kPermThreads) {
-            int32_t s = 0;
-            for (int w = 0; w < kPermThreads / 32; ++w) s += wcnt[w][ee];
-            running[ee] += s;
+            int32_t sum = 0;
+            for (int w = 0; w < kPermThreads / 32; ++w) {
+                const int32_t v = wcnt[w][ee];
+                if ((v >> 16) == r) sum += v & 0xffff;
+            }
+            running[cur ^ 1][ee] = running[cur][ee] + sum;
         }
         __syncthreads();
     }
 }
 
-// Plans of at most one block of slots (T*k <= 2048, e.g. decode batches): the
-// three steps above in one CTA and one launch, no workspace.
-__global__ void __launch_bounds__(kPermThreads) permute_single_kernel(
-    const int32_t* __restrict__ idx, int64_t n, int E, int32_t* __restrict__ counts,
+// ---------------------------------------------------------------------------
+// One-launch plan on a cluster (see the header comment).  CTA c of the
+// cluster owns slots [c * chunk, (c + 1) * chunk); ROUNDS * 1024 >= chunk.
+constexpr int kPcThreads = 1024;
+constexpr int kPcWarps = kPcThreads / 32;
+constexpr int kPcMaxCluster = 8;
+
+template <int ROUNDS>
+__global__ void __launch_bounds__(kPcThreads, 1) permute_cluster_kernel(
+    const int32_t* __restrict__ idx, int64_t n, int E, int64_t chunk, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
     int32_t* __restrict__ err_flag) {
     __shared__ int32_t hist[kMaxExperts];
-    __shared__ int32_t running[kMaxExperts];
-    __shared__ int32_t wcnt[kPermThreads / 32][kMaxExperts];
-    __shared__ int32_t warp_sum[kPermThreads / 32];
+    __shared__ int32_t running[2][kMaxExperts];
+    // per-warp counts of the current round, stamped with the round in the high
+    // half so that entries left from earlier rounds read as zero
+    __shared__ int32_t wcnt[kPcWarps][kMaxExperts];
+    __shared__ int32_t warp_sum[kPcWarps];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int e = tid; e < E; e += kPermThreads) hist[e] = 0;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int csize = static_cast<int>(gridDim.x);
+    const int64_t lo = rank * chunk;
+    const int64_t hi = lo + chunk < n ? lo + chunk : n;
+
+    for (int e = tid; e < E; e += kPcThreads) hist[e] = 0;
+    for (int i = tid; i < kPcWarps * kMaxExperts; i += kPcThreads)
+        (&wcnt[0][0])[i] = -1;                                  // stamp -1: no round
     __syncthreads();
+    // this thread's slots, one per round, kept in registers
+    int ev[ROUNDS];
     bool bad = false;
-    for (int r = 0; r < kPermRounds; ++r) {
-        const int64_t q = r * kPermThreads + tid;
-        if (q < n) {
-            const int e = idx[q];
-            if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
-            else bad = true;
+#pragma unroll
+    for (int r = 0; r < ROUNDS; ++r) {
+        const int64_t q = lo + static_cast<int64_t>(r) * kPcThreads + tid;
+        ev[r] = q < hi ? idx[q] : -1;
+    }
+#pragma unroll
+    for (int r = 0; r < ROUNDS; ++r) {
+        const int64_t q = lo + static_cast<int64_t>(r) * kPcThreads + tid;
+        if (q < hi) {
+            if (ev[r] >= 0 && ev[r] < E) atomicAdd(&hist[ev[r]], 1);
+            else { bad = true; ev[r] = -1; }
         }
     }
     if (bad) raise_error(err_flag, MOE_ERR_BAD_INDEX);
-    __syncthreads();
-    // exclusive scan of the counts (E <= 256 = blockDim)
-    const int32_t v = tid < E ? hist[tid] : 0;
-    int32_t incl = v;
+    cluster_sync();                                             // every CTA's hist is final
+
+    // per expert: total over the cluster and the count of the CTAs before this one
+    int32_t total = 0, before_cta = 0;
+    if (tid < E) {
+        const uint32_t local = smem_u32(&hist[tid]);
+        for (int c = 0; c < csize; ++c) {
+            int32_t v;
+            asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(mapa_shared(local, c))
+                         : "memory");
+            total += v;
+            if (c < rank) before_cta += v;
+        }
+    }
+    // exclusive scan of the totals over experts (E <= 256 < blockDim)
+    int32_t incl = total;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
@@ -155,43 +206,92 @@ __global__ void __launch_bounds__(kPermThreads) permute_single_kernel(
     }
     if (lane == 31) warp_sum[warp] = incl;
     __syncthreads();
-    int32_t before = 0;
-    for (int w = 0; w < warp; ++w) before += warp_sum[w];
     if (tid < E) {
-        const int32_t excl = before + incl - v;
-        counts[tid] = v;
-        offsets[tid] = excl;
-        running[tid] = excl;
-        if (tid == E - 1) offsets[E] = excl + v;
-    }
-    // stable scatter, rounds in slot order (as permute_scatter_kernel)
-    for (int r = 0; r < kPermRounds; ++r) {
-        for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads) wcnt[i / E][i % E] = 0;
-        __syncthreads();
-        const int64_t q = r * kPermThreads + tid;
-        int e = -1;
-        if (q < n) {
-            e = idx[q];
-            if (e < 0 || e >= E) e = -1;
+        int32_t excl = incl - total;
+        for (int w = 0; w < warp; ++w) excl += warp_sum[w];
+        running[0][tid] = excl + before_cta;
+        if (rank == 0) {
+            counts[tid] = total;
+            offsets[tid] = excl;
+            if (tid == E - 1) offsets[E] = excl + total;
         }
+    }
+    __syncthreads();
+
+    // stable scatter, rounds in slot order
+#pragma unroll
+    for (int r = 0; r < ROUNDS; ++r) {
+        const int cur = r & 1;
+        const int e = ev[r];
+        const int64_t q = lo + static_cast<int64_t>(r) * kPcThreads + tid;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int lane_rank = __popc(peers & ((1u << lane) - 1u));
-        if (e >= 0 && lane_rank == 0) wcnt[warp][e] = __popc(peers);
+        if (e >= 0 && lane_rank == 0) wcnt[warp][e] = (r << 16) | __popc(peers);
         __syncthreads();
         if (e >= 0) {
-            int32_t p = running[e] + lane_rank;
-            for (int w = 0; w < warp; ++w) p += wcnt[w][e];
+            int32_t p = running[cur][e] + lane_rank;
+            for (int w = 0; w < warp; ++w) {
+                const int32_t v = wcnt[w][e];
+                if ((v >> 16) == r) p += v & 0xffff;
+            }
             perm[p] = static_cast<int32_t>(q);
             inv[q] = p;
         }
-        __syncthreads();
-        for (int ee = tid; ee < E; ee += kPermThreads) {
-            int32_t s = 0;
-            for (int w = 0; w < kPermThreads / 32; ++w) s += wcnt[w][ee];
-            running[ee] += s;
+        for (int ee = tid; ee < E; ee += kPcThreads) {
+            int32_t sum = 0;
+            for (int w = 0; w < kPcWarps; ++w) {
+                const int32_t v = wcnt[w][ee];
+                if ((v >> 16) == r) sum += v & 0xffff;
+            }
+            running[cur ^ 1][ee] = running[cur][ee] + sum;
         }
         __syncthreads();
     }
+    cluster_sync();          // no CTA leaves while another may still read its hist
+}
+
+// Largest plan the one-launch cluster path takes.
+// (Beyond 8 rounds per CTA the three launches over many CTAs are faster.)
+constexpr int64_t kPcMaxSlots = static_cast<int64_t>(kPcMaxCluster) * 8 * kPcThreads;
+
+template <int ROUNDS>
+static cudaError_t launch_permute_cluster_t(const moe_shape& s, int csize, int64_t chunk,
+                                            const int32_t* idx, int32_t* counts, int32_t* offsets,
+                                            int32_t* perm, int32_t* inv, int32_t* err_flag,
+                                            cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(csize), 1, 1);
+    cfg.blockDim = dim3(kPcThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, permute_cluster_kernel<ROUNDS>, idx, s.T * s.k, s.E, chunk,
+                              counts, offsets, perm, inv, err_flag);
+}
+
+static cudaError_t launch_permute_cluster(const moe_shape& s, const int32_t* idx, int32_t* counts,
+                                          int32_t* offsets, int32_t* perm, int32_t* inv,
+                                          int32_t* err_flag, cudaStream_t st) {
+    const int64_t n = s.T * s.k;
+    int64_t csize = (n + kPcThreads - 1) / kPcThreads;
+    if (csize > kPcMaxCluster) csize = kPcMaxCluster;
+    if (csize < 1) csize = 1;
+    const int64_t chunk = (n + csize - 1) / csize;
+    const int64_t rounds = (chunk + kPcThreads - 1) / kPcThreads;
+    const int c = static_cast<int>(csize);
+    if (rounds <= 1)
+        return launch_permute_cluster_t<1>(s, c, chunk, idx, counts, offsets, perm, inv, err_flag, st);
+    if (rounds <= 2)
+        return launch_permute_cluster_t<2>(s, c, chunk, idx, counts, offsets, perm, inv, err_flag, st);
+    if (rounds <= 4)
+        return launch_permute_cluster_t<4>(s, c, chunk, idx, counts, offsets, perm, inv, err_flag, st);
+    return launch_permute_cluster_t<8>(s, c, chunk, idx, counts, offsets, perm, inv, err_flag, st);
 }
 
 size_t permute_workspace_bytes(const moe_shape& s) {
@@ -204,12 +304,9 @@ cudaError_t launch_permute(const moe_shape& s, const int32_t* idx, int32_t* coun
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* err_flag,
                            void* workspace, cudaStream_t st) {
     const int64_t n = s.T * s.k;
+    if (n <= kPcMaxSlots)
+        return launch_permute_cluster(s, idx, counts, offsets, perm, inv, err_flag, st);
     const int nblk = static_cast<int>((n + kPermSlotsPerBlock - 1) / kPermSlotsPerBlock);
-    if (nblk == 1) {
-        permute_single_kernel<<<1, kPermThreads, 0, st>>>(idx, n, s.E, counts, offsets, perm, inv,
-                                                          err_flag);
-        return cudaGetLastError();
-    }
     int32_t* blk = static_cast<int32_t*>(workspace);
     if (nblk > 0) {
         permute_hist_kernel<<<nblk, kPermThreads, 0, st>>>(idx, n, s.E, blk, err_flag);

@@ -221,3 +221,36 @@ def test_route_with_presplit_weight_matches_route(cuda_ok, cfg):
     assert float((a[1] - b[1]).abs().max()) <= 2 * tol
     for u, v in zip(b, c):
         assert torch.equal(u, v)
+
+
+@pytest.mark.parametrize("T,k,E,skew", [
+    (1, 1, 4, 0.0),            # one slot
+    (700, 1, 256, 0.0),        # E at its maximum, one CTA
+    (5001, 3, 64, 1.5),        # cluster of 8, two rounds, ragged last CTA, skewed
+    (8192, 2, 8, 0.0),         # the Mixtral-shaped plan: 8 CTAs x one round
+    (21845, 3, 16, 0.0),       # 65535 slots: the cluster path's largest plans (8 rounds)
+    (65537, 1, 32, 1.0),       # 65537 slots: above it, the three-launch path
+    (131073, 2, 64, 1.2),      # 262146 slots over 128 blocks
+])
+def test_permute_plans_match_the_oracle(cuda_ok, T, k, E, skew):
+    """counts, offsets, perm and inv bit-exact against the oracle's counting
+    sort, on random expert choices (skewed ones included)."""
+    import oracle
+    import sparse_mixture_experts_07_b200 as moe
+    rng = np.random.default_rng(T)
+    p = 1.0 / np.arange(1, E + 1) ** skew
+    idx = np.stack([rng.choice(E, size=k, replace=False, p=p / p.sum()) for _ in range(T)]) \
+        if T <= 5001 else rng.choice(E, size=(T, k), p=p / p.sum())
+    # top-k picks distinct experts per token; the plan itself does not need it
+    idx = idx.astype(np.int32)
+    shape = moe.Shape(T=T, H=128, I=128, E=E, k=k)
+    ws = moe.alloc_workspace(shape)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    counts, offsets, perm, inv = moe.permute(shape, torch.from_numpy(idx).cuda(), ws, err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    o_counts, o_offsets, o_perm, o_inv = oracle.permute(idx, E)
+    assert np.array_equal(counts.cpu().numpy(), o_counts)
+    assert np.array_equal(offsets.cpu().numpy(), o_offsets)
+    assert np.array_equal(perm.cpu().numpy(), o_perm)
+    assert np.array_equal(inv.cpu().numpy(), o_inv)
