@@ -22,16 +22,9 @@
 // every load is a contiguous 16 bytes: lane (g = lane/4, q = lane%4) loads
 // elements [base + 8q, base + 8q + 8) of weight rows g and g+8 and of token
 // row g, and feeds elements 0..3 to one MMA and 4..7 to the next.
-#include "common.cuh"
+#include "decode_common.cuh"
 
 namespace moe {
-
-namespace dec {
-constexpr int WARPS = 4;
-constexpr int THREADS = WARPS * 32;
-constexpr int MAX_ROWS = 8;      // rows per group handled here
-constexpr int UNROLL = 8;        // 32-element k-steps in flight per warp
-}  // namespace dec
 
 struct DecodeParams {
     const __nv_bfloat16* x;          // [T, H]
@@ -50,121 +43,11 @@ struct DecodeParams {
     float routed_scale;
 };
 
-// Active groups (routed experts with slots, then shared experts) and the
-// prefix of their work units.
-struct ActiveGroups {
-    int n;
-    int total_units;
-    int gid[kMaxGroups];
-    int unit_start[kMaxGroups + 1];
-};
-
-__device__ __forceinline__ void build_active(ActiveGroups& a, const DecodeParams& p, bool down) {
-    int n = 0, acc = 0;
-    for (int g = 0; g < p.E + p.S; ++g) {
-        const bool routed = g < p.E;
-        const int rows = routed ? p.offsets[g + 1] - p.offsets[g] : static_cast<int>(p.T);
-        if (rows <= 0) continue;
-        const int ncols = down ? p.H : (routed ? p.I : p.Is);
-        a.gid[n] = g;
-        a.unit_start[n] = acc;
-        acc += (ncols + 15) / 16;
-        ++n;
-    }
-    a.unit_start[n] = acc;
-    a.n = n;
-    a.total_units = acc;
-}
-
-__device__ __forceinline__ int find_active(const ActiveGroups& a, int unit) {
-    int lo = 0, hi = a.n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a.unit_start[mid] <= unit) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
-                                               uint32_t a2, uint32_t a3, uint32_t b0,
-                                               uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// c += W[rows w0 (g) and w1 (g+8)] . X[row xr]^T over one 32-element k-step,
-// given this lane's 16-byte pieces wa (row g), wb (row g+8), xv (token row g).
-__device__ __forceinline__ void mma_step(float (&c)[4], const uint4& wa, const uint4& wb,
-                                         const uint4& xv) {
-    mma_bf16_16816(c, wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
-    mma_bf16_16816(c, wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
-}
-
-// Predicated 16-byte loads (zero when !ok), written as volatile PTX so that
-// the compiler keeps them in program order ahead of the MMAs that consume
-// them: all loads of an unrolled step are in flight together.
-__device__ __forceinline__ uint4 ldg16(const __nv_bfloat16* p, bool ok) {
-    uint4 v;
-    asm volatile(
-        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-        "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
-        "@q ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
-        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-        : "l"(p), "r"(static_cast<int>(ok)));
-    return v;
-}
-
-// Same, for weights that are read once: do not allocate them in L1.
-__device__ __forceinline__ uint4 ldg16_stream(const __nv_bfloat16* p, bool ok) {
-    uint4 v;
-    asm volatile(
-        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-        "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
-        "@q ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
-        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-        : "l"(p), "r"(static_cast<int>(ok)));
-    return v;
-}
-
-// Element range [k0, k1) of warp w when K is split over the CTA's warps in
-// chunks of 32 * UNROLL elements (one unrolled loop iteration each).
-__device__ __forceinline__ void k_split(int K, int w, int& k0, int& k1) {
-    constexpr int CH = 32 * dec::UNROLL;
-    const int nchunks = (K + CH - 1) / CH;
-    k0 = ((nchunks * w) / dec::WARPS) * CH;
-    k1 = ((nchunks * (w + 1)) / dec::WARPS) * CH;
-}
-
-// Sums the WARPS partial fragments of a CTA: every warp writes its NF floats
-// per lane, then warp 0 reads all of them back.  Returns true in warp 0.
-template <int NF>
-__device__ __forceinline__ bool reduce_over_warps(float (&v)[NF], float* red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-    for (int j = 0; j < NF; ++j) red[(warp * NF + j) * 32 + lane] = v[j];
-    __syncthreads();
-    if (warp == 0) {
-#pragma unroll
-        for (int j = 0; j < NF; ++j) {
-            float acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < dec::WARPS; ++w) acc += red[(w * NF + j) * 32 + lane];
-            v[j] = acc;
-        }
-    }
-    __syncthreads();
-    return warp == 0;
-}
-
 // One CTA per work unit (grid-stride); its 4 warps split the contraction.
 __global__ void __launch_bounds__(dec::THREADS, 2) decode_gate_up_kernel(const DecodeParams p) {
     __shared__ ActiveGroups act;
     __shared__ float red[dec::WARPS * 8 * 32];
-    if (threadIdx.x == 0) build_active(act, p, false);
+    if (threadIdx.x == 0) build_active(act, p.offsets, p.E, p.S, p.T, p.I, p.Is);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     int s0, s1;
@@ -229,7 +112,7 @@ __global__ void __launch_bounds__(dec::THREADS, 2) decode_gate_up_kernel(const D
 __global__ void __launch_bounds__(dec::THREADS, 2) decode_down_kernel(const DecodeParams p) {
     __shared__ ActiveGroups act;
     __shared__ float red[dec::WARPS * 4 * 32];
-    if (threadIdx.x == 0) build_active(act, p, true);
+    if (threadIdx.x == 0) build_active(act, p.offsets, p.E, p.S, p.T, p.H, p.H);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int64_t routed_rows = p.T * p.k;

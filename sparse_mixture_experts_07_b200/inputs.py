@@ -222,3 +222,38 @@ def make_inputs(cfg: MoEConfig, seed: int = 0, weights_device: str = "cpu",
         "zipf_target": target,
         "redrawn_rows": redrawn,
     }
+
+
+# MXFP4 scale codes drawn for synthetic expert weights: 2^-8 or 2^-7.  With
+# codes uniform over the 16 E2M1 values (root mean square 2.93) the weights
+# then have a root mean square of about 0.018, near the initializer_range
+# (0.02) above.
+MXFP4_SCALE_CODES = (119, 120)
+
+
+def make_mxfp4_weights(cfg: MoEConfig, seed: int = 0, device: str = "cpu") -> dict:
+    """Routed expert weights in the MXFP4 storage layout, drawn at random.
+
+    gate_up_q [E, 2I, H/2] and down_q [E, H, I/2] are uniform random bytes (two
+    4-bit codes each); gate_up_s [E, 2I, H/32] and down_s [E, H, I/32] are drawn
+    uniformly from MXFP4_SCALE_CODES.  One generator on `device` seeded with
+    `seed` + 2, in that order.  H and I must be multiples of 32."""
+    E, H, I = cfg.E, cfg.H, cfg.I
+    if H % 32 or I % 32:
+        raise ValueError("MXFP4 weights need H and I to be multiples of 32")
+    g = torch.Generator(device=device).manual_seed(seed + 2)
+    codes = torch.tensor(MXFP4_SCALE_CODES, dtype=torch.uint8, device=device)
+
+    def qbytes(*shape):
+        return torch.randint(0, 256, shape, generator=g, dtype=torch.uint8, device=device)
+
+    def scales(*shape):
+        return codes[torch.randint(0, len(MXFP4_SCALE_CODES), shape, generator=g,
+                                   device=device)]
+
+    return {
+        "gate_up_q": qbytes(E, 2 * I, H // 2),
+        "gate_up_s": scales(E, 2 * I, H // 32),
+        "down_q": qbytes(E, H, I // 2),
+        "down_s": scales(E, H, I // 32),
+    }
