@@ -207,6 +207,33 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const int3
                        void* y_slots, int32_t* err_flag, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* moe_forward with the routed experts' weights in MXFP4, for decode batches
+ * ("Mixture of Experts in Transformers", section "from dense to sparse": at
+ * small batch the time is the bytes of the active experts' weights, and the
+ * gpt-oss experts are stored natively in mxfp4).  MXFP4 as the OCP
+ * Microscaling Formats v1.0 specification defines it: each block of 32
+ * consecutive weights along the contraction shares one E8M0 scale 2^(s-127)
+ * (255 = NaN); each weight is an FP4 E2M1 code (sign, 2-bit exponent with
+ * bias 1, 1-bit mantissa; values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives).
+ *   gate_up_q [E, 2I, H/2]  uint8, 16-byte aligned: weight 2j of a row in the
+ *                           low nibble of byte j, weight 2j+1 in the high
+ *                           nibble; rows [0, I) gate, [I, 2I) up
+ *   gate_up_s [E, 2I, H/32] uint8 E8M0 scale of each block of 32 weights
+ *   down_q    [E, H, I/2]   uint8, same packing;  down_s [E, H, I/32] uint8
+ * Other arguments, outputs and workspace as moe_forward (y_slots holds the
+ * T*k routed rows).  Supported: bf16 x, 1 <= T <= 8, no shared experts, H and
+ * I multiples of 32; otherwise MOE_ERR_UNSUPPORTED.  The products run in f16
+ * with float32 accumulation: each activation row (x, then h) is scaled by a
+ * power of two that puts its largest magnitude in [2^14, 2^15) and rounded to
+ * f16; the scaling is undone in float32.  Weights must stay below 2^128 in
+ * magnitude (scale codes up to 252). */
+MOE_API moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x,
+                                     const int32_t* offsets, const int32_t* perm,
+                                     const float* topk_w, const uint8_t* gate_up_q,
+                                     const uint8_t* gate_up_s, const uint8_t* down_q,
+                                     const uint8_t* down_s, void* y_slots, int32_t* err_flag,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* Combine ("Mixture of Experts in Transformers", expert backends: gather and
  * reorder the results).  y[t] = sum_j y_slots[inv[t*k+j]]
  *                               + sum_s y_slots[T*k + s*T + t],

@@ -75,15 +75,19 @@ def moe_block_mxfp4(x, w_router, router_bias, gate_up_q, gate_up_s, down_q, down
     xs = x.float().numpy() if hasattr(x, "float") else np.asarray(x, dtype=np.float64)
     gq, gs = np.asarray(gate_up_q), np.asarray(gate_up_s)
     dq, ds = np.asarray(down_q), np.asarray(down_s)
-    cache = {}
     y = np.zeros((len(toks), dq.shape[1]), dtype=np.float64)
-    for n, t in enumerate(toks):
+    # one expert's weights in memory at a time; each token still sums its k
+    # expert outputs in the order j = 0..k-1
+    outs = {}
+    for e in sorted(set(int(v) for v in idx.reshape(-1))):
+        # the values are exact in float32 (2-bit significands times 2^(s-127))
+        gu_e = dequantize(gq[e], gs[e]).astype(np.float32)
+        dn_e = dequantize(dq[e], ds[e]).astype(np.float32)
+        for n, t in enumerate(toks):
+            for j in range(k):
+                if int(idx[n, j]) == e:
+                    outs[(n, j)] = expert(gu_e, dn_e, xs[t].astype(np.float64))
+    for n in range(len(toks)):
         for j in range(k):
-            e = int(idx[n, j])
-            if e not in cache:
-                # the values are exact in float32 (2-bit significands times 2^(s-127))
-                cache[e] = (dequantize(gq[e], gs[e]).astype(np.float32),
-                            dequantize(dq[e], ds[e]).astype(np.float32))
-            gu_e, dn_e = cache[e]
-            y[n] += w[n, j] * expert(gu_e, dn_e, xs[t].astype(np.float64))
+            y[n] += w[n, j] * outs[(n, j)]
     return routed_scale * y, idx, w

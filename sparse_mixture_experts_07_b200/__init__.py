@@ -5,5 +5,5 @@ The kernels live in libmoe.so (CUDA for sm_100a, C ABI in include/moe.h);
 """
 from . import inputs  # noqa: F401
 from .moe import (MOE_BF16, MOE_F32, MoEError, MoELayer, Shape, alloc_workspace,  # noqa: F401
-                  combine, forward, load_library, permute, route, router_split,
+                  combine, forward, forward_mxfp4, load_library, permute, route, router_split,
                   workspace_size)

@@ -31,6 +31,10 @@ cudaError_t launch_ffn_sm100_pair(const moe_shape&, const void*, const void*, co
                                   const int32_t*, const float*, const void*, const void*,
                                   const void*, const void*, void*, void*, void*, int32_t*, int, int,
                                   cudaStream_t);
+cudaError_t launch_ffn_decode_mxfp4(const moe_shape&, const void*, const int32_t*,
+                                    const int32_t*, const float*, const uint8_t*, const uint8_t*,
+                                    const uint8_t*, const uint8_t*, void*, void*, int32_t*, void*,
+                                    int32_t*, void*, int, cudaStream_t);
 cudaError_t launch_combine(const moe_shape&, const void*, const int32_t*, void*, cudaStream_t);
 cudaError_t launch_gather_rows(const moe_shape&, const void*, const int32_t*, void*, int,
                                cudaStream_t);
@@ -77,7 +81,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 struct Workspace {
-    size_t permute_off, h_routed_off, h_shared_off, x_perm_off, total;
+    size_t permute_off, h_routed_off, h_shared_off, x_perm_off;
+    size_t mx_x16_off, mx_xexp_off, mx_h16_off, mx_hexp_off;   // MXFP4 decode (T <= 8)
+    size_t total;
 };
 
 Workspace layout(const moe_shape& s) {
@@ -93,6 +99,16 @@ Workspace layout(const moe_shape& s) {
     off += align_up(static_cast<size_t>(s.n_shared) * s.T * (s.n_shared ? s.I_shared : 0) * eb);
     w.x_perm_off = off;
     if (s.dtype == MOE_BF16) off += align_up(static_cast<size_t>(Tk) * s.H * 2);
+    if (s.dtype == MOE_BF16 && s.T <= 8) {
+        w.mx_x16_off = off;
+        off += align_up(static_cast<size_t>(s.T) * s.H * 2);
+        w.mx_xexp_off = off;
+        off += align_up(static_cast<size_t>(s.T) * 4);
+        w.mx_h16_off = off;
+        off += align_up(static_cast<size_t>(Tk) * s.I * 2);
+        w.mx_hexp_off = off;
+        off += align_up(static_cast<size_t>(Tk) * 4);
+    }
     w.total = off;
     return w;
 }
@@ -247,6 +263,34 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* off
     return cuda_status(moe::launch_ffn_sm100(s, x, x_perm, offsets, perm, topk_w, gate_up, down,
                                              sh_gate_up, sh_down, h_routed, h_shared, y_slots,
                                              err_flag, sms, 8, cs));
+}
+
+moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x, const int32_t* offsets,
+                             const int32_t* perm, const float* topk_w, const uint8_t* gate_up_q,
+                             const uint8_t* gate_up_s, const uint8_t* down_q,
+                             const uint8_t* down_s, void* y_slots, int32_t* err_flag,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    (void)err_flag;
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    const moe_shape& s = *shape;
+    if (s.T == 0) return MOE_OK;
+    if (s.dtype != MOE_BF16 || s.n_shared != 0 || s.T > 8 || s.H % 32 != 0 || s.I % 32 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (!x || !offsets || !perm || !topk_w || !gate_up_q || !gate_up_s || !down_q || !down_s ||
+        !y_slots)
+        return MOE_ERR_INVALID_ARG;
+    const Workspace w = layout(s);
+    if (!workspace || workspace_bytes < w.total) return MOE_ERR_WORKSPACE;
+    const void* ptrs[] = {x, gate_up_q, down_q, y_slots, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
+    char* ws = static_cast<char*>(workspace);
+    return cuda_status(moe::launch_ffn_decode_mxfp4(
+        s, x, offsets, perm, topk_w, gate_up_q, gate_up_s, down_q, down_s, ws + w.h_routed_off,
+        ws + w.mx_x16_off, reinterpret_cast<int32_t*>(ws + w.mx_xexp_off), ws + w.mx_h16_off,
+        reinterpret_cast<int32_t*>(ws + w.mx_hexp_off), y_slots, num_sms(),
+        static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* inv, void* y,

@@ -20,7 +20,8 @@ MOE_F32, MOE_BF16 = 0, 1
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_INDEX", 6: "MOE_ERR_TIMEOUT"}
 EXPORTS = ("moe_status_str", "moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
-           "moe_combine", "moe_router_split_size", "moe_router_split", "moe_route_split")
+           "moe_combine", "moe_router_split_size", "moe_router_split", "moe_route_split",
+           "moe_forward_mxfp4")
 
 
 class MoEShape(ctypes.Structure):
@@ -60,6 +61,7 @@ def load_library(path: str = LIB_PATH):
     lib.moe_router_split_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
     lib.moe_router_split.argtypes = [S, P, P, ctypes.c_size_t, P]
     lib.moe_route_split.argtypes = [S, P, P, P, P, P, P, P, P, P]
+    lib.moe_forward_mxfp4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     for f in EXPORTS[1:]:
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -190,6 +192,21 @@ def forward(shape: Shape, x, offsets, perm, topk_w, gate_up, down, sh_gate_up, s
     return y_slots
 
 
+def forward_mxfp4(shape: Shape, x, offsets, perm, topk_w, mxfp4: dict, workspace, err_flag,
+                  y_slots=None, stream=None):
+    """moe_forward with MXFP4 routed-expert weights (decode batches, T <= 8):
+    `mxfp4` holds gate_up_q, gate_up_s, down_q, down_s (uint8 device tensors)."""
+    lib = load_library()
+    if y_slots is None:
+        y_slots = torch.empty(shape.slot_rows, shape.H, dtype=shape.torch_dtype, device=x.device)
+    _check(lib.moe_forward_mxfp4(ctypes.byref(shape.c()), _ptr(x), _ptr(offsets), _ptr(perm),
+                                 _ptr(topk_w), _ptr(mxfp4["gate_up_q"]), _ptr(mxfp4["gate_up_s"]),
+                                 _ptr(mxfp4["down_q"]), _ptr(mxfp4["down_s"]), _ptr(y_slots),
+                                 _ptr(err_flag), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "moe_forward_mxfp4")
+    return y_slots
+
+
 def combine(shape: Shape, y_slots, inv, y=None, stream=None):
     """y [T, H] (dtype)."""
     lib = load_library()
@@ -208,15 +225,18 @@ class MoELayer:
     last call are kept in `self.last` for inspection.
     """
 
-    def __init__(self, shape: Shape, w_router, router_bias, gate_up, down, sh_gate_up=None,
-                 sh_down=None):
+    def __init__(self, shape: Shape, w_router, router_bias, gate_up=None, down=None,
+                 sh_gate_up=None, sh_down=None, mxfp4=None):
+        """Expert weights either as gate_up / down (dtype of `shape`), or as
+        `mxfp4` = {gate_up_q, gate_up_s, down_q, down_s} (decode batches)."""
         self.shape = shape
+        self.mxfp4 = mxfp4
         self.w_router, self.router_bias = w_router, router_bias
         # split once here, at load time; refresh it if w_router changes
         self.w_split = router_split(shape, w_router)
         self.gate_up, self.down = gate_up, down
         self.sh_gate_up, self.sh_down = sh_gate_up, sh_down
-        dev = gate_up.device
+        dev = (gate_up if mxfp4 is None else mxfp4["gate_up_q"]).device
         self.workspace = alloc_workspace(shape, dev)
         self.err_flag = torch.zeros(1, dtype=torch.int32, device=dev)
         T, k, E, H = shape.T, shape.k, shape.E, shape.H
@@ -238,8 +258,13 @@ class MoELayer:
                           err_flag=self.err_flag, w_split=self.w_split)
         counts, offsets, perm, inv = permute(s, idx, self.workspace, self.err_flag, out=b,
                                              stream=stream)
-        forward(s, x, offsets, perm, w, self.gate_up, self.down, self.sh_gate_up, self.sh_down,
-                self.workspace, self.err_flag, y_slots=b["y_slots"], stream=stream)
+        if self.mxfp4 is not None:
+            forward_mxfp4(s, x, offsets, perm, w, self.mxfp4, self.workspace, self.err_flag,
+                          y_slots=b["y_slots"], stream=stream)
+        else:
+            forward(s, x, offsets, perm, w, self.gate_up, self.down, self.sh_gate_up,
+                    self.sh_down, self.workspace, self.err_flag, y_slots=b["y_slots"],
+                    stream=stream)
         out = combine(s, b["y_slots"], inv, y=b["y"] if y is None else y, stream=stream)
         self.last = b
         return out

@@ -152,6 +152,27 @@ def test_router_split_argument_checks(lib):
                                None) == 2
 
 
+def test_forward_mxfp4_argument_checks(lib):
+    ok = ctypes.c_void_p(4096)
+    s = _shape(T=4, H=256, I=128)
+    _, need = _ws(lib, s)
+
+    def call(shape, ws_bytes=need, x=ok, q=ok, ws=ok):
+        return lib.moe_forward_mxfp4(ctypes.byref(shape), x, ok, ok, ok, q, ok, ok, ok, ok,
+                                     None, ws, ws_bytes, None)
+    assert call(_shape(T=9, H=256, I=128)) == 2              # decode batches only
+    assert call(_shape(T=4, H=256, I=128, n_shared=1, I_shared=64)) == 2
+    assert call(_shape(T=4, H=136, I=128)) == 2              # H not a multiple of 32
+    assert call(_shape(T=4, H=256, I=136)) == 2
+    assert call(_shape(T=4, H=256, I=128, dtype=moe.MOE_F32)) == 2
+    assert call(s, q=None) == 1
+    assert call(s, x=None) == 1
+    assert call(s, ws_bytes=need - 1) == 3
+    assert call(s, ws=None) == 3
+    assert call(s, x=ctypes.c_void_p(4096 + 8)) == 2
+    assert call(_shape(T=0, H=256, I=128), x=None, q=None, ws=None, ws_bytes=0) == 0
+
+
 def test_zero_tokens_is_a_no_op(lib):
     s = _shape(T=0)
     assert lib.moe_route(ctypes.byref(s), None, None, None, None, None, None, None, None) == 0
