@@ -59,6 +59,14 @@ struct GroupTableT {
     int32_t rows[MAXG];             // M of each group
     int32_t row0[MAXG];             // first row of the group in its A space
 };
+
+// All threads of the CTA copy offsets[0..E] into shared memory (one parallel
+// load instead of E dependent ones in the thread that builds a table); the
+// caller synchronises before the copy is read.
+__device__ __forceinline__ void stage_offsets(int32_t* dst, const int32_t* offsets, int E) {
+    for (int g = static_cast<int>(threadIdx.x); g <= E; g += static_cast<int>(blockDim.x))
+        dst[g] = offsets[g];
+}
 using GroupTable = GroupTableT<kMaxGroups>;
 
 // ---------------------------------------------------------------------------
@@ -314,10 +322,13 @@ namespace moe {
 // Builds the group table (one thread; at most kMaxGroups iterations).
 // Routed group g covers rows [offsets[g], offsets[g+1]); shared group E+s
 // covers the T token rows.  Tiles of a group: ceil(rows / BM) * n_tiles.
+// Built by one thread.  stage_offsets has put the routed experts' offsets in
+// gt.tile_start[0..E]; entry g is read (as offsets[g] and offsets[g+1]) before
+// the loop overwrites it with the tile prefix.
 template <int MAXG>
-__device__ __forceinline__ void build_group_table(GroupTableT<MAXG>& gt, const int32_t* offsets, int E,
-                                                  int S, int64_t T, int BM, int n_tiles_routed,
-                                                  int n_tiles_shared) {
+__device__ __forceinline__ void build_group_table(GroupTableT<MAXG>& gt, int E, int S, int64_t T,
+                                                  int BM, int n_tiles_routed, int n_tiles_shared) {
+    int32_t* offsets = gt.tile_start;
     int32_t acc = 0;
     gt.n_groups = E + S;
     for (int g = 0; g < E + S; ++g) {

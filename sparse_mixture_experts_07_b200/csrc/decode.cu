@@ -47,7 +47,9 @@ struct DecodeParams {
 __global__ void __launch_bounds__(dec::THREADS, 2) decode_gate_up_kernel(const DecodeParams p) {
     __shared__ ActiveGroups act;
     __shared__ float red[dec::WARPS * 8 * 32];
-    if (threadIdx.x == 0) build_active(act, p.offsets, p.E, p.S, p.T, p.I, p.Is);
+    stage_offsets(act.offs, p.offsets, p.E);
+    __syncthreads();
+    if (threadIdx.x == 0) build_active(act, p.E, p.S, p.T, p.I, p.Is);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     int s0, s1;
@@ -58,8 +60,8 @@ __global__ void __launch_bounds__(dec::THREADS, 2) decode_gate_up_kernel(const D
         const bool routed = grp < p.E;
         const int N = routed ? p.I : p.Is;
         const int i0 = (unit - act.unit_start[ai]) * 16;
-        const int rows = routed ? p.offsets[grp + 1] - p.offsets[grp] : static_cast<int>(p.T);
-        const int64_t row0 = routed ? p.offsets[grp] : static_cast<int64_t>(grp - p.E) * p.T;
+        const int rows = routed ? act.offs[grp + 1] - act.offs[grp] : static_cast<int>(p.T);
+        const int64_t row0 = routed ? act.offs[grp] : static_cast<int64_t>(grp - p.E) * p.T;
         const __nv_bfloat16* W =
             routed ? p.gate_up + static_cast<int64_t>(grp) * 2 * p.I * p.H
                    : p.sh_gate_up + static_cast<int64_t>(grp - p.E) * 2 * p.Is * p.H;
@@ -112,7 +114,9 @@ __global__ void __launch_bounds__(dec::THREADS, 2) decode_gate_up_kernel(const D
 __global__ void __launch_bounds__(dec::THREADS, 2) decode_down_kernel(const DecodeParams p) {
     __shared__ ActiveGroups act;
     __shared__ float red[dec::WARPS * 4 * 32];
-    if (threadIdx.x == 0) build_active(act, p.offsets, p.E, p.S, p.T, p.H, p.H);
+    stage_offsets(act.offs, p.offsets, p.E);
+    __syncthreads();
+    if (threadIdx.x == 0) build_active(act, p.E, p.S, p.T, p.H, p.H);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int64_t routed_rows = p.T * p.k;
@@ -124,8 +128,8 @@ __global__ void __launch_bounds__(dec::THREADS, 2) decode_down_kernel(const Deco
         int s0, s1;
         k_split(K, warp, s0, s1);
         const int n0 = (unit - act.unit_start[ai]) * 16;
-        const int rows = routed ? p.offsets[grp + 1] - p.offsets[grp] : static_cast<int>(p.T);
-        const int64_t row0 = routed ? p.offsets[grp] : static_cast<int64_t>(grp - p.E) * p.T;
+        const int rows = routed ? act.offs[grp + 1] - act.offs[grp] : static_cast<int>(p.T);
+        const int64_t row0 = routed ? act.offs[grp] : static_cast<int64_t>(grp - p.E) * p.T;
         const __nv_bfloat16* W = routed ? p.down + static_cast<int64_t>(grp) * p.H * p.I
                                         : p.sh_down + static_cast<int64_t>(grp - p.E) * p.H * p.Is;
         const __nv_bfloat16* hin = routed ? p.h_routed : p.h_shared;

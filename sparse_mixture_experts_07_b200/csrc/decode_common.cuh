@@ -22,13 +22,16 @@ struct ActiveGroups {
     int total_units;
     int gid[kMaxGroups];
     int unit_start[kMaxGroups + 1];
+    int32_t offs[kMaxExperts + 1];   // the routed experts' offsets (stage_offsets)
 };
 
 // Groups 0..E-1 are routed experts (rows from offsets), E..E+S-1 shared
 // experts (T rows each); a group's work units cover its ncols output
 // columns 16 at a time.
-__device__ __forceinline__ void build_active(ActiveGroups& a, const int32_t* offsets, int E, int S,
-                                             int64_t T, int ncols_routed, int ncols_shared) {
+// Built by one thread from a.offs, which stage_offsets filled.
+__device__ __forceinline__ void build_active(ActiveGroups& a, int E, int S, int64_t T,
+                                             int ncols_routed, int ncols_shared) {
+    const int32_t* offsets = a.offs;
     int n = 0, acc = 0;
     for (int g = 0; g < E + S; ++g) {
         const bool routed = g < E;

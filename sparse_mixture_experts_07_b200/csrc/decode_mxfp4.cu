@@ -11,29 +11,35 @@
 // Storage: q [rows, K/2] bytes, element 2j of a row in the low nibble of byte
 // j, element 2j+1 in the high nibble; s [rows, K/32] bytes.
 //
-// Same structure as the bf16 decode kernels (a CTA per (group, 16 output
-// rows), 4 warps splitting the contraction, mma.sync m16n8k16 with weight rows
-// as M and the group's <= 8 token rows as N), with three changes:
-//   - the products run in f16 x f16 -> f32: an E2M1 pair converts to an f16
-//     pair in one instruction (cvt.rn.f16x2.e2m1x2), exactly;
-//   - so the activations enter as f16: each row is multiplied by 2^-p first,
-//     p = floor(log2 max|row|) - 14, which puts the row's largest magnitude in
-//     [2^14, 2^15) (no overflow) and is undone in fp32 in the epilogue;
-//   - the contraction is permuted so that the 16 k-values of one MMA come from
-//     one block of each weight row: lane (g, q) reads bytes 4q..4q+3 of a
-//     block (weights 8q..8q+7), the first two bytes feed one MMA and the last
-//     two the next.  The two MMAs of a block accumulate from zero, and the
-//     block's scale multiplies the result into the fp32 accumulators (two
-//     scales per lane: weight rows g and g+8).
+// Work unit: (expert group, 16 output rows), as in the bf16 decode kernels;
+// the MMAs are mma.sync m16n8k16 with weight rows as M and the group's <= 8
+// token rows as N.  Per CTA:
+//   - warp 0 streams the unit's weight bytes through a ring of shared-memory
+//     stages: lane 0 issues, per weight matrix, MOE_MX_BOXES adjacent 16-row x
+//     128-byte TMA boxes (128-byte swizzle), so each row is read in runs of
+//     128 * MOE_MX_BOXES bytes; the 32 lanes store the stage's scales as
+//     floats, from scale bytes they loaded a few stages earlier (scale rows
+//     are not 16-byte aligned, so they cannot use TMA);
+//   - warps 1..MOE_MX_CONSUMERS split each stage's blocks, convert E2M1 pairs
+//     to f16 pairs (cvt.rn.f16x2.e2m1x2, exact) and run the MMAs in
+//     f16 x f16 -> f32; their partial sums meet in shared memory at the end
+//     of the unit.
+// Activations enter as f16: each row is multiplied by 2^-p first, p =
+// floor(log2 max|row|) - 14, which puts its largest magnitude in [2^14, 2^15);
+// the epilogue undoes it in fp32.  The contraction is permuted so that the 16
+// k-values of one MMA come from one block of each weight row: lane (g, q)
+// takes bytes 4q..4q+3 of a block (weights 8q..8q+7), the first two bytes
+// feed one MMA and the last two the next.  The two MMAs of a block start
+// from zero and the block's scale multiplies their sum into the fp32
+// accumulators.  Waits are bounded (MOE_ERR_TIMEOUT).
 #include "decode_common.cuh"
+#include "gemm_common.cuh"
 
 #include <cuda_fp16.h>
 
 namespace moe {
 
 namespace mx {
-constexpr int UNROLL_GU = 8;     // blocks in flight per lane, gate_up (4 weight rows)
-constexpr int UNROLL_DN = 16;    // blocks in flight per lane, down (2 weight rows)
 constexpr int PREP_THREADS = 256;
 }  // namespace mx
 
@@ -51,6 +57,7 @@ struct MxParams {
     const __half* h16;          // [T*k, I]  h * 2^-hexp[p]
     const int32_t* hexp;        // [T*k]
     __nv_bfloat16* y_slots;     // [T*k, H]
+    int32_t* err_flag;
     int64_t T;
     int H, I, E, k;
     float routed_scale;
@@ -113,16 +120,6 @@ __device__ __forceinline__ float e8m0_to_float(uint32_t s) {
                   : (s == 255 ? __uint_as_float(0x7fc00000u) : __uint_as_float(s << 23));
 }
 
-__device__ __forceinline__ uint32_t ldg_u32(const uint8_t* p, bool ok) {
-    uint32_t v;
-    asm volatile(
-        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\tmov.b32 %0, 0;\n\t"
-        "@q ld.global.nc.u32 %0, [%1];\n\t}"
-        : "=r"(v)
-        : "l"(p), "r"(static_cast<int>(ok)));
-    return v;
-}
-
 __device__ __forceinline__ uint32_t ldg_u8(const uint8_t* p, bool ok) {
     uint32_t v;
     asm volatile(
@@ -146,9 +143,9 @@ __device__ __forceinline__ uint4 ldg_v4(const void* p, bool ok) {
 
 // acc += scale(row g) / scale(row g+8) * (W_block . X_block) for one 32-weight
 // block: w0 / w1 are this lane's 4 bytes of rows g / g+8, xv its 8 f16 of the
-// token row, s0 / s1 the two rows' scale codes.
+// token row, f0 / f1 the two rows' block scales.
 __device__ __forceinline__ void mx_block(float (&acc)[4], uint32_t w0, uint32_t w1,
-                                         const uint4& xv, uint32_t s0, uint32_t s1) {
+                                         const uint4& xv, float f0, float f1) {
     uint32_t a[4], b[4];
     e2m1x8_to_f16(w0, a);
     e2m1x8_to_f16(w1, b);
@@ -156,151 +153,293 @@ __device__ __forceinline__ void mx_block(float (&acc)[4], uint32_t w0, uint32_t 
     float d[4];
     mma_f16_16816(d, a[0], b[0], a[1], b[1], xv.x, xv.y, zero);
     mma_f16_16816(d, a[2], b[2], a[3], b[3], xv.z, xv.w, d);
-    const float f0 = e8m0_to_float(s0), f1 = e8m0_to_float(s1);
     acc[0] = fmaf(f0, d[0], acc[0]);
     acc[1] = fmaf(f0, d[1], acc[1]);
     acc[2] = fmaf(f1, d[2], acc[2]);
     acc[3] = fmaf(f1, d[3], acc[3]);
 }
 
-// Blocks [b0, b1) of warp w when nblk blocks are split over the CTA's warps in
-// chunks of `unroll` blocks.
-__device__ __forceinline__ void block_split(int nblk, int unroll, int w, int& b0, int& b1) {
-    const int nchunks = (nblk + unroll - 1) / unroll;
-    b0 = ((nchunks * w) / dec::WARPS) * unroll;
-    b1 = ((nchunks * (w + 1)) / dec::WARPS) * unroll;
-    if (b1 > nblk) b1 = nblk;
+#ifndef MOE_MX_CONSUMERS
+#define MOE_MX_CONSUMERS 4
+#endif
+namespace mxt {
+constexpr int CONSUMERS = MOE_MX_CONSUMERS;     // warps 1..CONSUMERS
+constexpr int THREADS = 32 * (1 + CONSUMERS);
+constexpr int BOX_ROWS = 16;
+constexpr int BOX_BYTES = BOX_ROWS * 128;       // 16 rows x 8 blocks of 16 bytes
+constexpr int SMEM_BUDGET = 96 * 1024;          // ring bytes per CTA (two CTAs per SM)
+}  // namespace mxt
+
+#ifndef MOE_MX_BOXES
+#define MOE_MX_BOXES 4
+#endif
+
+// Stage geometry.  KIND 0: gate_up (K = H, output rows I; a stage holds NB
+// adjacent boxes of the 16 gate rows and NB of the matching 16 up rows).
+// KIND 1: down (K = I, output rows H; NB adjacent boxes of 16 rows).  A stage
+// covers BPS = 8 NB blocks of each weight row, so every row is read in runs of
+// 128 NB contiguous bytes.  Scale bytes of a stage: [R rows][BPS blocks].
+template <int KIND, int NB>
+struct MxGeo {
+    static constexpr int MAT = KIND == 0 ? 2 : 1;                // weight matrices per stage
+    static constexpr int BPS = 8 * NB;                           // blocks per stage
+    static constexpr int BPW = BPS / mxt::CONSUMERS;             // blocks per consumer warp
+    static constexpr int R = 16 * MAT;                           // weight rows per stage
+    static constexpr int Q_BYTES = MAT * NB * mxt::BOX_BYTES;    // a 1024-byte multiple
+    static constexpr int SC_BYTES = R * BPS * 4;                 // scales as float
+    static constexpr int NS = R * BPS / 32;                      // scales per producer lane
+    static constexpr int STAGES_FIT = mxt::SMEM_BUDGET / (Q_BYTES + SC_BYTES);
+    static constexpr int STAGES = STAGES_FIT < 4 ? 4 : (STAGES_FIT > 12 ? 12 : STAGES_FIT);
+    static constexpr int PREFETCH_FIT = 64 / NS;                 // stages of scales in registers
+    static constexpr int PREFETCH = PREFETCH_FIT < 2 ? 2 : (PREFETCH_FIT > 6 ? 6 : PREFETCH_FIT);
+    static constexpr int NF = KIND == 0 ? 8 : 4;                 // accumulators per lane
+    static constexpr int SMEM_BYTES = STAGES * (Q_BYTES + SC_BYTES) + 1024 + 2 * STAGES * 8 + 64;
+};
+
+template <int KIND, int NB>
+__global__ void __launch_bounds__(mxt::THREADS) decode_mx_kernel(
+    const __grid_constant__ CUtensorMap map_q, const MxParams p, uint64_t timeout_ns) {
+    using G = MxGeo<KIND, NB>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ ActiveGroups act;
+    __shared__ float red[mxt::CONSUMERS * G::NF * 32];
+    __shared__ int fail_sh;
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sc_ring = smem + G::STAGES * G::Q_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sc_ring + G::STAGES * G::SC_BYTES);
+    uint64_t* empty = full + G::STAGES;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t deadline = global_ns() + timeout_ns;
+
+    const int K = KIND == 0 ? p.H : p.I;                     // contraction
+    const int N = KIND == 0 ? p.I : p.H;                     // output rows per expert
+    const int64_t wrows = KIND == 0 ? 2 * static_cast<int64_t>(p.I) : p.H;   // weight rows per expert
+    const int nblk = K / 32;
+    const int nst = (nblk + G::BPS - 1) / G::BPS;            // stages per unit
+    const uint8_t* scales = KIND == 0 ? p.gu_s : p.dn_s;
+    const int64_t total_rows = static_cast<int64_t>(p.E) * wrows;
+
+    stage_offsets(act.offs, p.offsets, p.E);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        build_active(act, p.E, 0, p.T, N, N);
+        for (int s = 0; s < G::STAGES; ++s) {
+            mbar_init(&full[s], 1 + 32);           // TMA bytes + the 32 scale-copying lanes
+            mbar_init(&empty[s], mxt::CONSUMERS);
+        }
+        fail_sh = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&map_q);
+    }
+    __syncthreads();
+    const int n_units = act.total_units;
+    const int my_units = n_units > static_cast<int>(blockIdx.x)
+                             ? (n_units - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                             : 0;
+    const int total_f = my_units * nst;
+
+    // expert group and first output row of unit u
+    auto unit_row0 = [&](int u, int& grp, int& r0) {
+        const int ai = find_active(act, u);
+        grp = act.gid[ai];
+        r0 = (u - act.unit_start[ai]) * 16;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        // scale byte i = lane + 32 m of a stage: row i / BPS (KIND 0: gate rows
+        // 0-15, up rows 16-31), block i % BPS (consecutive lanes, consecutive
+        // blocks of one row: coalesced)
+        auto load_scales = [&](int f, uint32_t (&v)[G::NS]) {
+#pragma unroll
+            for (int m = 0; m < G::NS; ++m) v[m] = 0u;
+            if (f >= total_f) return;
+            const int u = static_cast<int>(blockIdx.x) + (f / nst) * static_cast<int>(gridDim.x);
+            const int st = f % nst;
+            int grp, r0;
+            unit_row0(u, grp, r0);
+            const int64_t base = static_cast<int64_t>(grp) * wrows + r0;
+#pragma unroll
+            for (int m = 0; m < G::NS; ++m) {
+                const int i = lane + 32 * m;
+                const int rr = i / G::BPS, blk = st * G::BPS + i % G::BPS;
+                const int64_t row = base + (KIND == 0 && rr >= 16 ? p.I + rr - 16 : rr);
+                v[m] = ldg_u8(scales + row * nblk + blk, row < total_rows && blk < nblk);
+            }
+        };
+        uint32_t sreg[G::PREFETCH][G::NS];
+#pragma unroll
+        for (int d = 0; d < G::PREFETCH; ++d) load_scales(d, sreg[d]);
+        bool ok = true;
+        for (int f0 = 0; f0 < total_f && ok; f0 += G::PREFETCH) {
+#pragma unroll
+            for (int d = 0; d < G::PREFETCH; ++d) {
+                const int f = f0 + d;
+                if (f >= total_f || !ok) break;
+                const int slot = f % G::STAGES;
+                const uint32_t ph = static_cast<uint32_t>(f / G::STAGES) & 1u;
+                if (!mbar_wait(&empty[slot], ph ^ 1u, deadline)) { ok = false; break; }
+                uint8_t* stage = smem + slot * G::Q_BYTES;
+                if (lane == 0) {
+                    const int u = static_cast<int>(blockIdx.x) + (f / nst) * static_cast<int>(gridDim.x);
+                    const int st = f % nst;
+                    int grp, r0;
+                    unit_row0(u, grp, r0);
+                    const int row = static_cast<int>(static_cast<int64_t>(grp) * wrows + r0);
+                    mbar_arrive_expect_tx(&full[slot], G::Q_BYTES);
+#pragma unroll
+                    for (int m = 0; m < G::MAT; ++m)
+#pragma unroll
+                        for (int b = 0; b < NB; ++b)
+                            tma_load_2d(stage + (m * NB + b) * mxt::BOX_BYTES, &map_q, &full[slot],
+                                        (st * NB + b) * 128, row + m * p.I);
+                }
+                float* sc = reinterpret_cast<float*>(sc_ring + slot * G::SC_BYTES);
+#pragma unroll
+                for (int m = 0; m < G::NS; ++m) sc[lane + 32 * m] = e8m0_to_float(sreg[d][m]);
+                mbar_arrive(&full[slot]);
+                load_scales(f + G::PREFETCH, sreg[d]);
+            }
+        }
+        if (!ok) raise_error(p.err_flag, MOE_ERR_TIMEOUT);
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int cw = warp - 1, g = lane >> 2, q = lane & 3;
+    bool ok = true;
+    int f = 0;
+    for (int ui = 0; ui < my_units; ++ui) {
+        const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
+        int grp, r0;
+        unit_row0(u, grp, r0);
+        const int rows = act.offs[grp + 1] - act.offs[grp];
+        const int64_t row0 = act.offs[grp];
+        const bool tok_ok = g < rows;
+        const __half* brow;                       // this lane's token row (column g)
+        if (KIND == 0) {
+            const int64_t tok = tok_ok ? p.perm[row0 + g] / p.k : 0;
+            brow = p.x16 + tok * p.H;
+        } else {
+            brow = p.h16 + (row0 + (tok_ok ? g : 0)) * p.I;
+        }
+        // epilogue factors of this lane's two token columns (2q, 2q+1), fetched
+        // now so that their latency hides under the unit's stages
+        float un[2] = {1.f, 1.f}, wsc[2] = {0.f, 0.f};
+        if (cw == 0) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int t = 2 * q + c;
+                if (t < rows) {
+                    if (KIND == 0) {
+                        const int64_t tk = p.perm[row0 + t] / p.k;
+                        un[c] = __uint_as_float(static_cast<uint32_t>(127 + p.xexp[tk]) << 23);
+                    } else {
+                        un[c] = __uint_as_float(static_cast<uint32_t>(127 + p.hexp[row0 + t]) << 23);
+                        wsc[c] = p.routed_scale * p.topk_w[p.perm[row0 + t]];
+                    }
+                }
+            }
+        }
+        float acc[G::NF];
+#pragma unroll
+        for (int j = 0; j < G::NF; ++j) acc[j] = 0.f;
+        // this warp's activation fragments, loaded one stage ahead of their use
+        auto load_b = [&](int st, uint4 (&v)[G::BPW]) {
+#pragma unroll
+            for (int i = 0; i < G::BPW; ++i) {
+                const int blk = st * G::BPS + cw * G::BPW + i;
+                v[i] = ldg_v4(brow + blk * 32 + 8 * q, tok_ok && st < nst && blk < nblk);
+            }
+        };
+        uint4 bv[G::BPW], bn[G::BPW];
+        load_b(0, bv);
+        for (int st = 0; st < nst; ++st, ++f) {
+            const int slot = f % G::STAGES;
+            const uint32_t ph = static_cast<uint32_t>(f / G::STAGES) & 1u;
+            load_b(st + 1, bn);
+            if (ok && !mbar_wait(&full[slot], ph, deadline)) ok = false;
+            const uint8_t* stage = smem + slot * G::Q_BYTES;
+            const float* sc = reinterpret_cast<const float*>(sc_ring + slot * G::SC_BYTES);
+#pragma unroll
+            for (int i = 0; i < G::BPW; ++i) {
+                const int jj = cw * G::BPW + i;                  // block within the stage
+                const uint8_t* bx = stage + (jj >> 3) * mxt::BOX_BYTES;
+                const uint32_t swz = static_cast<uint32_t>(((jj & 7) ^ g) << 4) + 4 * q;
+                const uint32_t w0 = *reinterpret_cast<const uint32_t*>(bx + g * 128 + swz);
+                const uint32_t w1 = *reinterpret_cast<const uint32_t*>(bx + (g + 8) * 128 + swz);
+                if (KIND == 0) {
+                    const uint8_t* ux = bx + NB * mxt::BOX_BYTES;
+                    const uint32_t v0 = *reinterpret_cast<const uint32_t*>(ux + g * 128 + swz);
+                    const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ux + (g + 8) * 128 + swz);
+                    float tg[4] = {acc[0], acc[1], acc[2], acc[3]};
+                    float tu[4] = {acc[4], acc[5], acc[6], acc[7]};
+                    mx_block(tg, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
+                    mx_block(tu, v0, v1, bv[i], sc[(16 + g) * G::BPS + jj],
+                             sc[(24 + g) * G::BPS + jj]);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) { acc[j] = tg[j]; acc[4 + j] = tu[j]; }
+                } else {
+                    float t4[4] = {acc[0], acc[1], acc[2], acc[3]};
+                    mx_block(t4, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[j] = t4[j];
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+#pragma unroll
+            for (int i = 0; i < G::BPW; ++i) bv[i] = bn[i];
+        }
+        // partial sums of the four consumer warps meet in shared memory
+#pragma unroll
+        for (int j = 0; j < G::NF; ++j) red[(cw * G::NF + j) * 32 + lane] = acc[j];
+        if (!ok) fail_sh = 1;
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * mxt::CONSUMERS) : "memory");
+        if (cw == 0) {
+#pragma unroll
+            for (int j = 0; j < G::NF; ++j) {
+                float v = 0.f;
+#pragma unroll
+                for (int w = 0; w < mxt::CONSUMERS; ++w) v += red[(w * G::NF + j) * 32 + lane];
+                acc[j] = v;
+            }
+            // acc[0], acc[1]: weight row g, tokens 2q, 2q+1; acc[2], acc[3]: row g+8
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = (j < 2) ? g : g + 8;
+                const int t = 2 * q + (j & 1);
+                if (t < rows && r0 + r < N && ok) {
+                    if (KIND == 0) {
+                        const float gv = acc[j] * un[j & 1];
+                        const float h = gv / (1.f + __expf(-gv)) * (acc[4 + j] * un[j & 1]);
+                        p.h[(row0 + t) * p.I + r0 + r] = __float2bfloat16_rn(h);
+                    } else {
+                        p.y_slots[(row0 + t) * p.H + r0 + r] =
+                            __float2bfloat16_rn(wsc[j & 1] * un[j & 1] * acc[j]);
+                    }
+                }
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * mxt::CONSUMERS) : "memory");
+        if (fail_sh) break;
+    }
+    if (cw == 0 && lane == 0 && !ok) raise_error(p.err_flag, MOE_ERR_TIMEOUT);
 }
 
-__global__ void __launch_bounds__(dec::THREADS, 2) decode_mx_gate_up_kernel(const MxParams p) {
-    __shared__ ActiveGroups act;
-    __shared__ float red[dec::WARPS * 8 * 32];
-    if (threadIdx.x == 0) build_active(act, p.offsets, p.E, 0, p.T, p.I, p.I);
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int nblk = p.H / 32;
-    int bs0, bs1;
-    block_split(nblk, mx::UNROLL_GU, warp, bs0, bs1);
-    const int64_t qrow = p.H / 2, srow = p.H / 32;
-    for (int unit = blockIdx.x; unit < act.total_units; unit += gridDim.x) {
-        const int ai = find_active(act, unit);
-        const int grp = act.gid[ai];
-        const int i0 = (unit - act.unit_start[ai]) * 16;
-        const int rows = p.offsets[grp + 1] - p.offsets[grp];
-        const int64_t row0 = p.offsets[grp];
-        const bool tok_ok = g < rows;
-        const int64_t tok = tok_ok ? p.perm[row0 + g] / p.k : 0;
-        const __half* xrow = p.x16 + tok * p.H;
-        const bool r0_ok = i0 + g < p.I, r1_ok = i0 + g + 8 < p.I;
-        const int64_t wr = static_cast<int64_t>(grp) * 2 * p.I + i0 + g;   // gate row g
-        const uint8_t* qg0 = p.gu_q + wr * qrow + 4 * q;
-        const uint8_t* qg1 = qg0 + 8 * qrow;
-        const uint8_t* qu0 = qg0 + static_cast<int64_t>(p.I) * qrow;
-        const uint8_t* qu1 = qg1 + static_cast<int64_t>(p.I) * qrow;
-        const uint8_t* sg0 = p.gu_s + wr * srow;
-        const uint8_t* sg1 = sg0 + 8 * srow;
-        const uint8_t* su0 = sg0 + static_cast<int64_t>(p.I) * srow;
-        const uint8_t* su1 = sg1 + static_cast<int64_t>(p.I) * srow;
-        float cg[4] = {0.f, 0.f, 0.f, 0.f}, cu[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int b = bs0; b < bs1; b += mx::UNROLL_GU) {
-            uint32_t wg0[mx::UNROLL_GU], wg1[mx::UNROLL_GU], wu0[mx::UNROLL_GU], wu1[mx::UNROLL_GU];
-            uint32_t tg0[mx::UNROLL_GU], tg1[mx::UNROLL_GU], tu0[mx::UNROLL_GU], tu1[mx::UNROLL_GU];
-            uint4 xv[mx::UNROLL_GU];
-#pragma unroll
-            for (int u = 0; u < mx::UNROLL_GU; ++u) {
-                const int blk = b + u;
-                const bool in = blk < bs1;
-                const int64_t qo = static_cast<int64_t>(blk) * 16;
-                wg0[u] = ldg_u32(qg0 + qo, in && r0_ok);
-                wg1[u] = ldg_u32(qg1 + qo, in && r1_ok);
-                wu0[u] = ldg_u32(qu0 + qo, in && r0_ok);
-                wu1[u] = ldg_u32(qu1 + qo, in && r1_ok);
-                tg0[u] = ldg_u8(sg0 + blk, in && r0_ok);
-                tg1[u] = ldg_u8(sg1 + blk, in && r1_ok);
-                tu0[u] = ldg_u8(su0 + blk, in && r0_ok);
-                tu1[u] = ldg_u8(su1 + blk, in && r1_ok);
-                xv[u] = ldg_v4(xrow + blk * 32 + 8 * q, in && tok_ok);
-            }
-#pragma unroll
-            for (int u = 0; u < mx::UNROLL_GU; ++u) {
-                mx_block(cg, wg0[u], wg1[u], xv[u], tg0[u], tg1[u]);
-                mx_block(cu, wu0[u], wu1[u], xv[u], tu0[u], tu1[u]);
-            }
-        }
-        float c[8] = {cg[0], cg[1], cg[2], cg[3], cu[0], cu[1], cu[2], cu[3]};
-        if (!reduce_over_warps<8>(c, red)) continue;
-        // c[0], c[1]: weight row g, tokens 2q, 2q+1; c[2], c[3]: row g+8 (up at +4)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int r = (j < 2) ? g : g + 8;
-            const int t = 2 * q + (j & 1);
-            if (t < rows && i0 + r < p.I) {
-                const int64_t tk = p.perm[row0 + t] / p.k;
-                const float up_scale = __uint_as_float(static_cast<uint32_t>(127 + p.xexp[tk]) << 23);
-                const float gv = c[j] * up_scale;
-                const float h = gv / (1.f + __expf(-gv)) * (c[4 + j] * up_scale);
-                p.h[(row0 + t) * p.I + i0 + r] = __float2bfloat16_rn(h);
-            }
-        }
-    }
-}
-
-__global__ void __launch_bounds__(dec::THREADS, 2) decode_mx_down_kernel(const MxParams p) {
-    __shared__ ActiveGroups act;
-    __shared__ float red[dec::WARPS * 4 * 32];
-    if (threadIdx.x == 0) build_active(act, p.offsets, p.E, 0, p.T, p.H, p.H);
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int nblk = p.I / 32;
-    int bs0, bs1;
-    block_split(nblk, mx::UNROLL_DN, warp, bs0, bs1);
-    const int64_t qrow = p.I / 2, srow = p.I / 32;
-    for (int unit = blockIdx.x; unit < act.total_units; unit += gridDim.x) {
-        const int ai = find_active(act, unit);
-        const int grp = act.gid[ai];
-        const int n0 = (unit - act.unit_start[ai]) * 16;
-        const int rows = p.offsets[grp + 1] - p.offsets[grp];
-        const int64_t row0 = p.offsets[grp];
-        const bool tok_ok = g < rows;
-        const __half* hrow = p.h16 + (row0 + (tok_ok ? g : 0)) * p.I;
-        const bool r0_ok = n0 + g < p.H, r1_ok = n0 + g + 8 < p.H;
-        const int64_t wr = static_cast<int64_t>(grp) * p.H + n0 + g;
-        const uint8_t* q0 = p.dn_q + wr * qrow + 4 * q;
-        const uint8_t* q1 = q0 + 8 * qrow;
-        const uint8_t* s0 = p.dn_s + wr * srow;
-        const uint8_t* s1 = s0 + 8 * srow;
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int b = bs0; b < bs1; b += mx::UNROLL_DN) {
-            uint32_t w0[mx::UNROLL_DN], w1[mx::UNROLL_DN], t0[mx::UNROLL_DN], t1[mx::UNROLL_DN];
-            uint4 hv[mx::UNROLL_DN];
-#pragma unroll
-            for (int u = 0; u < mx::UNROLL_DN; ++u) {
-                const int blk = b + u;
-                const bool in = blk < bs1;
-                const int64_t qo = static_cast<int64_t>(blk) * 16;
-                w0[u] = ldg_u32(q0 + qo, in && r0_ok);
-                w1[u] = ldg_u32(q1 + qo, in && r1_ok);
-                t0[u] = ldg_u8(s0 + blk, in && r0_ok);
-                t1[u] = ldg_u8(s1 + blk, in && r1_ok);
-                hv[u] = ldg_v4(hrow + blk * 32 + 8 * q, in && tok_ok);
-            }
-#pragma unroll
-            for (int u = 0; u < mx::UNROLL_DN; ++u) mx_block(c, w0[u], w1[u], hv[u], t0[u], t1[u]);
-        }
-        if (!reduce_over_warps<4>(c, red)) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int r = (j < 2) ? g : g + 8;
-            const int t = 2 * q + (j & 1);
-            if (t < rows && n0 + r < p.H) {
-                const int64_t orow = row0 + t;
-                const float unscale =
-                    __uint_as_float(static_cast<uint32_t>(127 + p.hexp[orow]) << 23);
-                const float scale = p.routed_scale * p.topk_w[p.perm[orow]] * unscale;
-                p.y_slots[orow * p.H + n0 + r] = __float2bfloat16_rn(scale * c[j]);
-            }
-        }
-    }
+// uint8 2D [rows, cols] map, box 128 columns x 16 rows, 128-byte swizzle.
+static bool make_map_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc || rows <= 0 || cols <= 0) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(mxt::BOX_ROWS)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // moe_forward_mxfp4: T <= 8, bf16 activations, routed experts only.
@@ -308,8 +447,8 @@ cudaError_t launch_ffn_decode_mxfp4(const moe_shape& s, const void* x, const int
                                     const int32_t* perm, const float* topk_w,
                                     const uint8_t* gu_q, const uint8_t* gu_s, const uint8_t* dn_q,
                                     const uint8_t* dn_s, void* h, void* x16, int32_t* xexp,
-                                    void* h16, int32_t* hexp, void* y_slots, int num_sms,
-                                    cudaStream_t st) {
+                                    void* h16, int32_t* hexp, void* y_slots, int32_t* err_flag,
+                                    int num_sms, cudaStream_t st) {
     if (s.T > dec::MAX_ROWS || s.T < 1 || s.dtype != MOE_BF16 || s.n_shared != 0 ||
         s.H % 32 != 0 || s.I % 32 != 0)
         return cudaErrorInvalidValue;
@@ -327,25 +466,44 @@ cudaError_t launch_ffn_decode_mxfp4(const moe_shape& s, const void* x, const int
     p.h16 = static_cast<const __half*>(h16);
     p.hexp = hexp;
     p.y_slots = static_cast<__nv_bfloat16*>(y_slots);
+    p.err_flag = err_flag;
     p.T = s.T;
     p.H = s.H;
     p.I = s.I;
     p.E = s.E;
     p.k = s.k;
     p.routed_scale = s.routed_scale;
-    const int grid = num_sms * 4;
+    CUtensorMap map_gu, map_dn;
+    if (!make_map_u8(&map_gu, gu_q, static_cast<int64_t>(s.E) * 2 * s.I, s.H / 2) ||
+        !make_map_u8(&map_dn, dn_q, static_cast<int64_t>(s.E) * s.H, s.I / 2))
+        return cudaErrorInvalidValue;
+    using G0 = MxGeo<0, MOE_MX_BOXES>;
+    using G1 = MxGeo<1, MOE_MX_BOXES>;
+    cudaError_t e = cudaFuncSetAttribute(decode_mx_kernel<0, MOE_MX_BOXES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         G0::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_mx_kernel<1, MOE_MX_BOXES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, G1::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // as many CTAs as fit next to each other (shared memory), on every SM
+    const int grid0 = num_sms * ((200 * 1024) / G0::SMEM_BYTES);
+    const int grid1 = num_sms * ((200 * 1024) / G1::SMEM_BYTES);
+    const uint64_t timeout = 4000000000ull;
     rows_to_f16_kernel<<<static_cast<unsigned>(s.T), mx::PREP_THREADS, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<__half*>(x16), xexp, s.H);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_mx_gate_up_kernel<<<grid, dec::THREADS, 0, st>>>(p);
+    decode_mx_kernel<0, MOE_MX_BOXES><<<grid0, mxt::THREADS, G0::SMEM_BYTES, st>>>(map_gu, p,
+                                                                                   timeout);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     rows_to_f16_kernel<<<static_cast<unsigned>(s.T * s.k), mx::PREP_THREADS, 0, st>>>(
         static_cast<const __nv_bfloat16*>(h), static_cast<__half*>(h16), hexp, s.I);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_mx_down_kernel<<<grid, dec::THREADS, 0, st>>>(p);
+    decode_mx_kernel<1, MOE_MX_BOXES><<<grid1, mxt::THREADS, G1::SMEM_BYTES, st>>>(map_dn, p,
+                                                                                   timeout);
     return cudaGetLastError();
 }
 

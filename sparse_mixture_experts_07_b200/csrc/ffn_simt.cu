@@ -43,8 +43,9 @@ __global__ void __launch_bounds__(256) simt_gate_up_kernel(SimtArgs a) {
     __shared__ float Bg[kSimtBN][kSimtBK + 1];
     __shared__ float Bu[kSimtBN][kSimtBK + 1];
     __shared__ int64_t arow[kSimtBM];
-    if (threadIdx.x == 0)
-        build_group_table(gt, a.offsets, a.E, a.S, a.T, kSimtBM, 1, 1);
+    stage_offsets(gt.tile_start, a.offsets, a.E);
+    __syncthreads();
+    if (threadIdx.x == 0) build_group_table(gt, a.E, a.S, a.T, kSimtBM, 1, 1);
     __syncthreads();
     const int tile = blockIdx.x;
     if (tile >= gt.total_tiles) return;
@@ -110,8 +111,9 @@ __global__ void __launch_bounds__(256) simt_down_kernel(SimtArgs a) {
     __shared__ GroupTable gt;
     __shared__ float As[kSimtBM][kSimtBK + 1];
     __shared__ float Bd[kSimtBN][kSimtBK + 1];
-    if (threadIdx.x == 0)
-        build_group_table(gt, a.offsets, a.E, a.S, a.T, kSimtBM, 1, 1);
+    stage_offsets(gt.tile_start, a.offsets, a.E);
+    __syncthreads();
+    if (threadIdx.x == 0) build_group_table(gt, a.E, a.S, a.T, kSimtBM, 1, 1);
     __syncthreads();
     const int tile = blockIdx.x;
     if (tile >= gt.total_tiles) return;

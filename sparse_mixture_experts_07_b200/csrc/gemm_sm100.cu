@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
     const uint64_t deadline = global_ns() + p.timeout_ns;
     constexpr int n_cols_per_tile = (EPI == kSwiGLU) ? BN / 2 : BN;
 
+    stage_offsets(gt.tile_start, p.offsets, p.E);
+    __syncthreads();
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
         mbar_init(drain, 1);
         abort_sh = 0;
         fence_barrier_init();
-        build_group_table(gt, p.offsets, p.E, p.S, p.T, BM, p.n_tiles_routed, p.n_tiles_shared);
+        build_group_table(gt, p.E, p.S, p.T, BM, p.n_tiles_routed, p.n_tiles_shared);
         tma_prefetch_desc(&map_a_routed);
         tma_prefetch_desc(&map_b_routed);
         if (p.S > 0) {

@@ -34,7 +34,7 @@ cudaError_t launch_ffn_sm100_pair(const moe_shape&, const void*, const void*, co
 cudaError_t launch_ffn_decode_mxfp4(const moe_shape&, const void*, const int32_t*,
                                     const int32_t*, const float*, const uint8_t*, const uint8_t*,
                                     const uint8_t*, const uint8_t*, void*, void*, int32_t*, void*,
-                                    int32_t*, void*, int, cudaStream_t);
+                                    int32_t*, void*, int32_t*, int, cudaStream_t);
 cudaError_t launch_combine(const moe_shape&, const void*, const int32_t*, void*, cudaStream_t);
 cudaError_t launch_gather_rows(const moe_shape&, const void*, const int32_t*, void*, int,
                                cudaStream_t);
@@ -270,7 +270,6 @@ moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x, const int32_
                              const uint8_t* gate_up_s, const uint8_t* down_q,
                              const uint8_t* down_s, void* y_slots, int32_t* err_flag,
                              void* workspace, size_t workspace_bytes, void* stream) {
-    (void)err_flag;
     moe_status st = check_shape(shape);
     if (st != MOE_OK) return st;
     const moe_shape& s = *shape;
@@ -289,7 +288,7 @@ moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x, const int32_
     return cuda_status(moe::launch_ffn_decode_mxfp4(
         s, x, offsets, perm, topk_w, gate_up_q, gate_up_s, down_q, down_s, ws + w.h_routed_off,
         ws + w.mx_x16_off, reinterpret_cast<int32_t*>(ws + w.mx_xexp_off), ws + w.mx_h16_off,
-        reinterpret_cast<int32_t*>(ws + w.mx_hexp_off), y_slots, num_sms(),
+        reinterpret_cast<int32_t*>(ws + w.mx_hexp_off), y_slots, err_flag, num_sms(),
         static_cast<cudaStream_t>(stream)));
 }
 
