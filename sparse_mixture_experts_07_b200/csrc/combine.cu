@@ -93,9 +93,60 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
          i += static_cast<int64_t>(gridDim.x) * 256) {
         const int64_t p = i / vec_per_row;
         const int v = static_cast<int>(i - p * vec_per_row);
-        const int64_t t = perm[p] / k;
-        x_perm[i] = x[t * vec_per_row + v];
+        const int64_t q = perm[p];
+        if (q >= 0 && q < n_rows) x_perm[i] = x[(q / k) * vec_per_row + v];
     }
+}
+
+// inv[perm[p]] = p: the sorted position of every slot.
+__global__ void __launch_bounds__(256) invert_perm_kernel(const int32_t* __restrict__ perm,
+                                                          int32_t* __restrict__ inv, int64_t n) {
+    for (int64_t p = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; p < n;
+         p += static_cast<int64_t>(gridDim.x) * 256) {
+        const int32_t q = perm[p];
+        // a plan with skipped slots (bad expert index) leaves holes: stay in bounds
+        if (q >= 0 && q < n) inv[q] = static_cast<int32_t>(p);
+    }
+}
+
+// Token-major gather: thread i reads the 16-byte piece i of x once and writes
+// it to the k sorted rows of that token, x_perm[inv[t*k + j]] (bf16, H % 8 == 0).
+// x is read from memory once even when it does not fit in L2.
+__global__ void __launch_bounds__(256) gather_by_token_kernel(const uint4* __restrict__ x,
+                                                              const int32_t* __restrict__ inv,
+                                                              uint4* __restrict__ x_perm,
+                                                              int64_t n_tokens, int vec_per_row,
+                                                              int k) {
+    const int64_t total = n_tokens * vec_per_row;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * 256) {
+        const int64_t t = i / vec_per_row;
+        const int v = static_cast<int>(i - t * vec_per_row);
+        const uint4 val = x[i];
+        for (int j = 0; j < k; ++j) {
+            const int64_t p = inv[t * k + j];
+            if (p >= 0 && p < n_tokens * k) x_perm[p * vec_per_row + v] = val;
+        }
+    }
+}
+
+cudaError_t launch_gather_by_token(const moe_shape& s, const void* x, const int32_t* perm,
+                                   int32_t* inv_scratch, void* x_perm, int num_sms,
+                                   cudaStream_t st) {
+    const int64_t n = s.T * s.k;
+    int64_t grid = (n + 255) / 256;
+    if (grid > static_cast<int64_t>(num_sms) * 8) grid = static_cast<int64_t>(num_sms) * 8;
+    if (grid < 1) return cudaSuccess;
+    invert_perm_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(perm, inv_scratch, n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int vpr = s.H / 8;
+    const int64_t total = s.T * vpr;
+    grid = (total + 255) / 256;
+    if (grid > static_cast<int64_t>(num_sms) * 16) grid = static_cast<int64_t>(num_sms) * 16;
+    gather_by_token_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
+        static_cast<const uint4*>(x), inv_scratch, static_cast<uint4*>(x_perm), s.T, vpr, s.k);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const moe_shape& s, const void* x, const int32_t* perm,

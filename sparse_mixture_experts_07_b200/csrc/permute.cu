@@ -59,10 +59,18 @@ __global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(
     const int e = threadIdx.x;
     int32_t run = 0;
     if (e < E) {
-        for (int b = 0; b < nblk; ++b) {
-            const int32_t c = blk[static_cast<int64_t>(b) * E + e];
-            blk[static_cast<int64_t>(b) * E + e] = run;
-            run += c;
+        // 16 independent loads in flight, then their running prefix
+        constexpr int B = 16;
+        for (int b0 = 0; b0 < nblk; b0 += B) {
+            int32_t c[B];
+#pragma unroll
+            for (int j = 0; j < B; ++j)
+                c[j] = b0 + j < nblk ? blk[static_cast<int64_t>(b0 + j) * E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < B; ++j) {
+                if (b0 + j < nblk) blk[static_cast<int64_t>(b0 + j) * E + e] = run;
+                run += c[j];
+            }
         }
         counts[e] = run;
     }
