@@ -17,13 +17,14 @@
 //   - warp 0 streams the unit's weight bytes through a ring of shared-memory
 //     stages: lane 0 issues, per weight matrix, MOE_MX_BOXES adjacent 16-row x
 //     128-byte TMA boxes (128-byte swizzle), so each row is read in runs of
-//     128 * MOE_MX_BOXES bytes; the 32 lanes store the stage's scales as
-//     floats, from scale bytes they loaded a few stages earlier (scale rows
-//     are not 16-byte aligned, so they cannot use TMA);
-//   - warps 1..MOE_MX_CONSUMERS split each stage's blocks, convert E2M1 pairs
-//     to f16 pairs (cvt.rn.f16x2.e2m1x2, exact) and run the MMAs in
-//     f16 x f16 -> f32; their partial sums meet in shared memory at the end
-//     of the unit.
+//     128 * MOE_MX_BOXES bytes;
+//   - warps 1..MOE_MX_CONSUMERS split each stage's blocks; each lane loads the
+//     block scales of its weight rows and its activation fragments one stage
+//     ahead (scale rows are not 16-byte aligned, so they cannot use TMA),
+//     converts E2M1 pairs to f16 pairs (cvt.rn.f16x2.e2m1x2, exact) and runs
+//     the MMAs in f16 x f16 -> f32; the warps' partial sums meet in shared
+//     memory at the end of the unit.  (With MOE_MX_CONSUMER_SCALES 0 the
+//     producer warp copies the scales into the ring instead, as floats.)
 // Activations enter as f16: each row is multiplied by 2^-p first, p =
 // floor(log2 max|row|) - 14, which puts its largest magnitude in [2^14, 2^15);
 // the epilogue undoes it in fp32.  The contraction is permuted so that the 16
@@ -167,11 +168,20 @@ constexpr int CONSUMERS = MOE_MX_CONSUMERS;     // warps 1..CONSUMERS
 constexpr int THREADS = 32 * (1 + CONSUMERS);
 constexpr int BOX_ROWS = 16;
 constexpr int BOX_BYTES = BOX_ROWS * 128;       // 16 rows x 8 blocks of 16 bytes
-constexpr int SMEM_BUDGET = 96 * 1024;          // ring bytes per CTA (two CTAs per SM)
+#ifndef MOE_MX_RING_KB
+#define MOE_MX_RING_KB 64
+#endif
+constexpr int SMEM_BUDGET = MOE_MX_RING_KB * 1024;   // ring bytes per CTA
 }  // namespace mxt
 
 #ifndef MOE_MX_BOXES
-#define MOE_MX_BOXES 4
+#define MOE_MX_BOXES 2
+#endif
+#ifndef MOE_MX_CONSUMER_SCALES
+#define MOE_MX_CONSUMER_SCALES 1
+#endif
+#ifndef MOE_MX_MIN_BLOCKS
+#define MOE_MX_MIN_BLOCKS 3
 #endif
 
 // Stage geometry.  KIND 0: gate_up (K = H, output rows I; a stage holds NB
@@ -186,10 +196,10 @@ struct MxGeo {
     static constexpr int BPW = BPS / mxt::CONSUMERS;             // blocks per consumer warp
     static constexpr int R = 16 * MAT;                           // weight rows per stage
     static constexpr int Q_BYTES = MAT * NB * mxt::BOX_BYTES;    // a 1024-byte multiple
-    static constexpr int SC_BYTES = R * BPS * 4;                 // scales as float
+    static constexpr int SC_BYTES = MOE_MX_CONSUMER_SCALES ? 0 : R * BPS * 4;   // scales as float
     static constexpr int NS = R * BPS / 32;                      // scales per producer lane
     static constexpr int STAGES_FIT = mxt::SMEM_BUDGET / (Q_BYTES + SC_BYTES);
-    static constexpr int STAGES = STAGES_FIT < 4 ? 4 : (STAGES_FIT > 12 ? 12 : STAGES_FIT);
+    static constexpr int STAGES = STAGES_FIT < 4 ? 4 : (STAGES_FIT > 24 ? 24 : STAGES_FIT);
     static constexpr int PREFETCH_FIT = 64 / NS;                 // stages of scales in registers
     static constexpr int PREFETCH = PREFETCH_FIT < 2 ? 2 : (PREFETCH_FIT > 6 ? 6 : PREFETCH_FIT);
     static constexpr int NF = KIND == 0 ? 8 : 4;                 // accumulators per lane
@@ -197,7 +207,7 @@ struct MxGeo {
 };
 
 template <int KIND, int NB>
-__global__ void __launch_bounds__(mxt::THREADS) decode_mx_kernel(
+__global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_kernel(
     const __grid_constant__ CUtensorMap map_q, const MxParams p, uint64_t timeout_ns) {
     using G = MxGeo<KIND, NB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -225,7 +235,8 @@ __global__ void __launch_bounds__(mxt::THREADS) decode_mx_kernel(
     if (threadIdx.x == 0) {
         build_active(act, p.E, 0, p.T, N, N);
         for (int s = 0; s < G::STAGES; ++s) {
-            mbar_init(&full[s], 1 + 32);           // TMA bytes + the 32 scale-copying lanes
+            // TMA bytes (+ the 32 scale-copying lanes when the producer copies scales)
+            mbar_init(&full[s], MOE_MX_CONSUMER_SCALES ? 1 : 1 + 32);
             mbar_init(&empty[s], mxt::CONSUMERS);
         }
         fail_sh = 0;
@@ -246,6 +257,34 @@ __global__ void __launch_bounds__(mxt::THREADS) decode_mx_kernel(
         r0 = (u - act.unit_start[ai]) * 16;
     };
 
+    if (warp == 0 && MOE_MX_CONSUMER_SCALES) {
+        // ------------------------------------------------------------ producer
+        // lane 0 alone: the weight boxes of every stage, the unit looked up once
+        if (lane != 0) return;
+        bool ok = true;
+        int f = 0;
+        for (int ui = 0; ui < my_units && ok; ++ui) {
+            const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
+            int grp, r0;
+            unit_row0(u, grp, r0);
+            const int row = static_cast<int>(static_cast<int64_t>(grp) * wrows + r0);
+            for (int st = 0; st < nst; ++st, ++f) {
+                const int slot = f % G::STAGES;
+                const uint32_t ph = static_cast<uint32_t>(f / G::STAGES) & 1u;
+                if (!mbar_wait(&empty[slot], ph ^ 1u, deadline)) { ok = false; break; }
+                uint8_t* stage = smem + slot * G::Q_BYTES;
+                mbar_arrive_expect_tx(&full[slot], G::Q_BYTES);
+#pragma unroll
+                for (int m = 0; m < G::MAT; ++m)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+                        tma_load_2d(stage + (m * NB + b) * mxt::BOX_BYTES, &map_q, &full[slot],
+                                    (st * NB + b) * 128, row + m * p.I);
+            }
+        }
+        if (!ok) raise_error(p.err_flag, MOE_ERR_TIMEOUT);
+        return;
+    }
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         // scale byte i = lane + 32 m of a stage: row i / BPS (KIND 0: gate rows
@@ -355,10 +394,38 @@ __global__ void __launch_bounds__(mxt::THREADS) decode_mx_kernel(
         };
         uint4 bv[G::BPW], bn[G::BPW];
         load_b(0, bv);
+        // block scales of this lane's weight rows (g, g+8; KIND 0 also the up
+        // rows), loaded by the consumers one stage ahead when the producer does
+        // not stage them
+        constexpr int SR = KIND == 0 ? 4 : 2;
+        const uint8_t* srow[SR];
+        bool sok[SR];
+        {
+            const int64_t wr0 = static_cast<int64_t>(grp) * wrows + r0 + g;
+#pragma unroll
+            for (int r = 0; r < SR; ++r) {
+                const int64_t row = wr0 + (r & 1) * 8 + (r >= 2 ? p.I : 0);
+                sok[r] = row < total_rows;
+                srow[r] = scales + (sok[r] ? row : 0) * nblk;
+            }
+        }
+        auto load_s = [&](int st, uint32_t (&v)[G::BPW][SR]) {
+            if (!MOE_MX_CONSUMER_SCALES) return;
+#pragma unroll
+            for (int i = 0; i < G::BPW; ++i) {
+                const int blk = st * G::BPS + cw * G::BPW + i;
+#pragma unroll
+                for (int r = 0; r < SR; ++r)
+                    v[i][r] = ldg_u8(srow[r] + blk, sok[r] && st < nst && blk < nblk);
+            }
+        };
+        uint32_t sv[G::BPW][SR], sn[G::BPW][SR];
+        load_s(0, sv);
         for (int st = 0; st < nst; ++st, ++f) {
             const int slot = f % G::STAGES;
             const uint32_t ph = static_cast<uint32_t>(f / G::STAGES) & 1u;
             load_b(st + 1, bn);
+            load_s(st + 1, sn);
             if (ok && !mbar_wait(&full[slot], ph, deadline)) ok = false;
             const uint8_t* stage = smem + slot * G::Q_BYTES;
             const float* sc = reinterpret_cast<const float*>(sc_ring + slot * G::SC_BYTES);
@@ -375,14 +442,25 @@ __global__ void __launch_bounds__(mxt::THREADS) decode_mx_kernel(
                     const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ux + (g + 8) * 128 + swz);
                     float tg[4] = {acc[0], acc[1], acc[2], acc[3]};
                     float tu[4] = {acc[4], acc[5], acc[6], acc[7]};
-                    mx_block(tg, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
-                    mx_block(tu, v0, v1, bv[i], sc[(16 + g) * G::BPS + jj],
-                             sc[(24 + g) * G::BPS + jj]);
+                    if (MOE_MX_CONSUMER_SCALES) {
+                        mx_block(tg, w0, w1, bv[i], e8m0_to_float(sv[i][0]),
+                                 e8m0_to_float(sv[i][1]));
+                        mx_block(tu, v0, v1, bv[i], e8m0_to_float(sv[i][2]),
+                                 e8m0_to_float(sv[i][3]));
+                    } else {
+                        mx_block(tg, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
+                        mx_block(tu, v0, v1, bv[i], sc[(16 + g) * G::BPS + jj],
+                                 sc[(24 + g) * G::BPS + jj]);
+                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j) { acc[j] = tg[j]; acc[4 + j] = tu[j]; }
                 } else {
                     float t4[4] = {acc[0], acc[1], acc[2], acc[3]};
-                    mx_block(t4, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
+                    if (MOE_MX_CONSUMER_SCALES)
+                        mx_block(t4, w0, w1, bv[i], e8m0_to_float(sv[i][0]),
+                                 e8m0_to_float(sv[i][SR - 1]));
+                    else
+                        mx_block(t4, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) acc[j] = t4[j];
                 }
@@ -390,7 +468,11 @@ __global__ void __launch_bounds__(mxt::THREADS) decode_mx_kernel(
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
 #pragma unroll
-            for (int i = 0; i < G::BPW; ++i) bv[i] = bn[i];
+            for (int i = 0; i < G::BPW; ++i) {
+                bv[i] = bn[i];
+#pragma unroll
+                for (int r = 0; r < SR; ++r) sv[i][r] = sn[i][r];
+            }
         }
         // partial sums of the four consumer warps meet in shared memory
 #pragma unroll
@@ -487,8 +569,9 @@ cudaError_t launch_ffn_decode_mxfp4(const moe_shape& s, const void* x, const int
                              cudaFuncAttributeMaxDynamicSharedMemorySize, G1::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // as many CTAs as fit next to each other (shared memory), on every SM
-    const int grid0 = num_sms * ((200 * 1024) / G0::SMEM_BYTES);
-    const int grid1 = num_sms * ((200 * 1024) / G1::SMEM_BYTES);
+    const int per_sm0 = (200 * 1024) / G0::SMEM_BYTES, per_sm1 = (200 * 1024) / G1::SMEM_BYTES;
+    const int grid0 = num_sms * (per_sm0 > 0 ? per_sm0 : 1);
+    const int grid1 = num_sms * (per_sm1 > 0 ? per_sm1 : 1);
     const uint64_t timeout = 4000000000ull;
     rows_to_f16_kernel<<<static_cast<unsigned>(s.T), mx::PREP_THREADS, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<__half*>(x16), xexp, s.H);
