@@ -164,12 +164,14 @@ def host_inputs(inp: dict) -> dict:
     return {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
 
 
-def bytes_decode(cfg, counts) -> float:
+def bytes_decode(cfg, counts, mxfp4: bool = False) -> float:
     """Algorithmic HBM bytes of one decode step: the touched experts' weights
-    once, the router weight, x in, y out, and the slot buffer written and read."""
+    once (MXFP4: half a byte per weight plus one scale byte per 32), the router
+    weight, x in, y out, and the slot buffer written and read."""
     eb = 2 if cfg.dtype == "bf16" else 4
+    wb = 0.5 + 1.0 / 32.0 if mxfp4 else eb
     active = int((counts > 0).sum())
-    w = active * 3 * cfg.H * cfg.I * eb + cfg.n_shared * 3 * cfg.H * cfg.I_shared * eb
+    w = active * 3 * cfg.H * cfg.I * wb + cfg.n_shared * 3 * cfg.H * cfg.I_shared * eb
     return w + cfg.E * cfg.H * 4 + 2 * cfg.T * cfg.H * eb + \
         2 * cfg.T * (cfg.k + cfg.n_shared) * cfg.H * eb
 
@@ -198,7 +200,9 @@ def run_reference(args, cfg, rank, world):
         "data": "synthetic (seeded; shapes of the named model, random-init weights)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E,
                    "k": cfg.k, "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
-                   "routed_scale": cfg.routed_scale, "storage": cfg.dtype},
+                   "routed_scale": cfg.routed_scale,
+                   "weights": "mxfp4 (E2M1 codes, E8M0 scales per 32)" if mx is not None
+                              else cfg.dtype, "storage": cfg.dtype},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"each step: the block for {samples[-1]} random tokens of the "
                                    f"{cfg.T}-token batch (full routing of those tokens, all their "
@@ -234,8 +238,14 @@ def run_cuda(args, cfg, rank, local, world):
     inp = make_inputs(cfg, seed=rank, weights_device=str(dev))
     shape = moe.Shape.from_config(cfg)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    layer = moe.MoELayer(shape, d["w_router"], d["router_bias"], d["gate_up"], d["down"],
-                         d["sh_gate_up"], d["sh_down"])
+    mx = None
+    if args.weights == "mxfp4":
+        from sparse_mixture_experts_07_b200.inputs import make_mxfp4_weights
+        mx = make_mxfp4_weights(cfg, seed=rank, device=str(dev))
+        layer = moe.MoELayer(shape, d["w_router"], d["router_bias"], mxfp4=mx)
+    else:
+        layer = moe.MoELayer(shape, d["w_router"], d["router_bias"], d["gate_up"], d["down"],
+                             d["sh_gate_up"], d["sh_down"])
     x = d["x"]
     stream = torch.cuda.current_stream(dev)
 
@@ -264,9 +274,13 @@ def run_cuda(args, cfg, rank, local, world):
                                   err_flag=layer.err_flag)
             moe.permute(shape, idx, layer.workspace, layer.err_flag, out=b)
             fwd_start[i].record(stream)
-            moe.forward(shape, x, b["offsets"], b["perm"], w, layer.gate_up, layer.down,
-                        layer.sh_gate_up, layer.sh_down, layer.workspace, layer.err_flag,
-                        y_slots=b["y_slots"])
+            if mx is not None:
+                moe.forward_mxfp4(shape, x, b["offsets"], b["perm"], w, mx, layer.workspace,
+                                  layer.err_flag, y_slots=b["y_slots"])
+            else:
+                moe.forward(shape, x, b["offsets"], b["perm"], w, layer.gate_up, layer.down,
+                            layer.sh_gate_up, layer.sh_down, layer.workspace, layer.err_flag,
+                            y_slots=b["y_slots"])
             fwd_end[i].record(stream)
             moe.combine(shape, b["y_slots"], b["inv"], y=b["y"])
         s1.record(stream)
@@ -340,11 +354,12 @@ def run_cuda(args, cfg, rank, local, world):
         if os.path.exists(src) and tr.get("sha") == src_sha(src):
             traffic = tr["bytes"]
     if decode:
-        algo = bytes_decode(cfg, counts)
+        algo = bytes_decode(cfg, counts, mxfp4=mx is not None)
         achieved = algo / (fwd_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "moe_forward (expert FFN launches)",
+                "kernel": "moe_forward_mxfp4 (f16 prep + MXFP4 expert FFN launches)"
+                          if mx is not None else "moe_forward (expert FFN launches)",
                 "peak_kind": f"{peaks['source']} HBM copy"}
     else:
         flops = 2.0 * cfg.T * (3 * cfg.k * cfg.H * cfg.I + 3 * cfg.n_shared * cfg.I_shared * cfg.H)
@@ -359,18 +374,24 @@ def run_cuda(args, cfg, rank, local, world):
                 "peak_kind": f"{peaks['source']} bf16 {'sustained' if long_run else 'burst'}",
                 "frac_of_burst": achieved / peaks["bf16_tflops"]}
 
+    if mx is not None:
+        weight_bytes = sum(v.numel() for v in mx.values())
+    else:
+        weight_bytes = (inp["gate_up"].numel() + inp["down"].numel()) * eb
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16" if mx is not None else ("bf16" if cfg.dtype == "bf16" else "f32"),
         "data": "synthetic (seeded; shapes of the named model, random-init weights)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E,
                    "k": cfg.k, "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
                    "routed_scale": cfg.routed_scale,
+                   "weights": "mxfp4 (E2M1 codes, E8M0 scales per 32)" if mx is not None
+                              else cfg.dtype,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (expert weights "
-                         f"{(inp['gate_up'].numel() + inp['down'].numel()) * eb / 1e9:.2f} GB "
-                         "streamed every step)"},
+                         f"{weight_bytes / 1e9:.2f} GB streamed every step)"},
         "tflops": 2.0 * cfg.T * (cfg.H * cfg.E + 3 * cfg.k * cfg.H * cfg.I +
                                  3 * cfg.n_shared * cfg.I_shared * cfg.H) * args.steps * world /
                   (ms_total / 1000.0) / 1e12,
@@ -381,7 +402,23 @@ def run_cuda(args, cfg, rank, local, world):
         "clocks": clk.summary(),
         "expert_counts": counts.tolist(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and mx is not None:
+        # the oracle's MXFP4 block on the whole (decode) batch: dequantise the
+        # selected experts, then the float64 expert math
+        import oracle
+        from oracle import mxfp4 as oracle_mx
+        host = host_inputs(inp)
+        hm = {k: v.cpu() for k, v in mx.items()}
+        t0 = time.perf_counter()
+        oracle_mx.moe_block_mxfp4(host["x"], host["w_router"], host["router_bias"],
+                                  hm["gate_up_q"], hm["gate_up_s"], hm["down_q"], hm["down_s"],
+                                  k=cfg.k, routed_scale=cfg.routed_scale)
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {
+            "value": cfg.T / el, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"the MXFP4 block for all {cfg.T} tokens ({el:.1f} s: numpy dequantisation "
+                      "of the selected experts, then float64 expert math)"}
+    elif rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = host_inputs(inp)
         r, n, el, cores = cpu_oracle_rate(cfg, host)
         line["cpu_baseline"] = {
@@ -401,8 +438,12 @@ def main():
     ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"],
+                    help="expert weight format; mxfp4 runs the decode path (T <= 8)")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
+    if args.weights == "mxfp4" and not (cfg.T <= 8 and cfg.dtype == "bf16" and cfg.n_shared == 0):
+        ap.error("--weights mxfp4 needs a bf16 decode configuration (T <= 8, no shared experts)")
     rank, local, world = dist_setup()
     try:
         if args.impl == "reference":
