@@ -4,6 +4,8 @@ TEST INFRASTRUCTURE.  Only tests/, __graft_entry__.smoke() and bench.py's
 CPU-baseline leg may import this package.  The CUDA implementation never does.
 The arithmetic lives in moe_oracle.c, which carries the definitions and the
 passages of the pages each step follows; this file only marshals arguments.
+`oracle.mxfp4` (numpy) decodes MXFP4 expert weights and feeds them to the
+same expert arithmetic.
 
 Functions accept torch CPU tensors (float32, or bfloat16 for activations and
 expert weights) or numpy arrays, and return numpy arrays (float64 results).

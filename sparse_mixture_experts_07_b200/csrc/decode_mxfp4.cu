@@ -23,8 +23,7 @@
 //     ahead (scale rows are not 16-byte aligned, so they cannot use TMA),
 //     converts E2M1 pairs to f16 pairs (cvt.rn.f16x2.e2m1x2, exact) and runs
 //     the MMAs in f16 x f16 -> f32; the warps' partial sums meet in shared
-//     memory at the end of the unit.  (With MOE_MX_CONSUMER_SCALES 0 the
-//     producer warp copies the scales into the ring instead, as floats.)
+//     memory at the end of the unit.
 // Activations enter as f16: each row is multiplied by 2^-p first, p =
 // floor(log2 max|row|) - 14, which puts its largest magnitude in [2^14, 2^15);
 // the epilogue undoes it in fp32.  The contraction is permuted so that the 16
@@ -177,9 +176,6 @@ constexpr int SMEM_BUDGET = MOE_MX_RING_KB * 1024;   // ring bytes per CTA
 #ifndef MOE_MX_BOXES
 #define MOE_MX_BOXES 2
 #endif
-#ifndef MOE_MX_CONSUMER_SCALES
-#define MOE_MX_CONSUMER_SCALES 1
-#endif
 #ifndef MOE_MX_MIN_BLOCKS
 #define MOE_MX_MIN_BLOCKS 3
 #endif
@@ -196,14 +192,11 @@ struct MxGeo {
     static constexpr int BPW = BPS / mxt::CONSUMERS;             // blocks per consumer warp
     static constexpr int R = 16 * MAT;                           // weight rows per stage
     static constexpr int Q_BYTES = MAT * NB * mxt::BOX_BYTES;    // a 1024-byte multiple
-    static constexpr int SC_BYTES = MOE_MX_CONSUMER_SCALES ? 0 : R * BPS * 4;   // scales as float
-    static constexpr int NS = R * BPS / 32;                      // scales per producer lane
-    static constexpr int STAGES_FIT = mxt::SMEM_BUDGET / (Q_BYTES + SC_BYTES);
+    static constexpr int SR = 2 * MAT;                           // scale rows per lane
+    static constexpr int STAGES_FIT = mxt::SMEM_BUDGET / Q_BYTES;
     static constexpr int STAGES = STAGES_FIT < 4 ? 4 : (STAGES_FIT > 24 ? 24 : STAGES_FIT);
-    static constexpr int PREFETCH_FIT = 64 / NS;                 // stages of scales in registers
-    static constexpr int PREFETCH = PREFETCH_FIT < 2 ? 2 : (PREFETCH_FIT > 6 ? 6 : PREFETCH_FIT);
     static constexpr int NF = KIND == 0 ? 8 : 4;                 // accumulators per lane
-    static constexpr int SMEM_BYTES = STAGES * (Q_BYTES + SC_BYTES) + 1024 + 2 * STAGES * 8 + 64;
+    static constexpr int SMEM_BYTES = STAGES * Q_BYTES + 1024 + 2 * STAGES * 8 + 64;
 };
 
 template <int KIND, int NB>
@@ -216,8 +209,7 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
     __shared__ int fail_sh;
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* sc_ring = smem + G::STAGES * G::Q_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sc_ring + G::STAGES * G::SC_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::Q_BYTES);
     uint64_t* empty = full + G::STAGES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t deadline = global_ns() + timeout_ns;
@@ -235,8 +227,7 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
     if (threadIdx.x == 0) {
         build_active(act, p.E, 0, p.T, N, N);
         for (int s = 0; s < G::STAGES; ++s) {
-            // TMA bytes (+ the 32 scale-copying lanes when the producer copies scales)
-            mbar_init(&full[s], MOE_MX_CONSUMER_SCALES ? 1 : 1 + 32);
+            mbar_init(&full[s], 1);                // one arrive.expect_tx per stage
             mbar_init(&empty[s], mxt::CONSUMERS);
         }
         fail_sh = 0;
@@ -248,7 +239,6 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
     const int my_units = n_units > static_cast<int>(blockIdx.x)
                              ? (n_units - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
                              : 0;
-    const int total_f = my_units * nst;
 
     // expert group and first output row of unit u
     auto unit_row0 = [&](int u, int& grp, int& r0) {
@@ -257,7 +247,7 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
         r0 = (u - act.unit_start[ai]) * 16;
     };
 
-    if (warp == 0 && MOE_MX_CONSUMER_SCALES) {
+    if (warp == 0) {
         // ------------------------------------------------------------ producer
         // lane 0 alone: the weight boxes of every stage, the unit looked up once
         if (lane != 0) return;
@@ -285,66 +275,6 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
         if (!ok) raise_error(p.err_flag, MOE_ERR_TIMEOUT);
         return;
     }
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        // scale byte i = lane + 32 m of a stage: row i / BPS (KIND 0: gate rows
-        // 0-15, up rows 16-31), block i % BPS (consecutive lanes, consecutive
-        // blocks of one row: coalesced)
-        auto load_scales = [&](int f, uint32_t (&v)[G::NS]) {
-#pragma unroll
-            for (int m = 0; m < G::NS; ++m) v[m] = 0u;
-            if (f >= total_f) return;
-            const int u = static_cast<int>(blockIdx.x) + (f / nst) * static_cast<int>(gridDim.x);
-            const int st = f % nst;
-            int grp, r0;
-            unit_row0(u, grp, r0);
-            const int64_t base = static_cast<int64_t>(grp) * wrows + r0;
-#pragma unroll
-            for (int m = 0; m < G::NS; ++m) {
-                const int i = lane + 32 * m;
-                const int rr = i / G::BPS, blk = st * G::BPS + i % G::BPS;
-                const int64_t row = base + (KIND == 0 && rr >= 16 ? p.I + rr - 16 : rr);
-                v[m] = ldg_u8(scales + row * nblk + blk, row < total_rows && blk < nblk);
-            }
-        };
-        uint32_t sreg[G::PREFETCH][G::NS];
-#pragma unroll
-        for (int d = 0; d < G::PREFETCH; ++d) load_scales(d, sreg[d]);
-        bool ok = true;
-        for (int f0 = 0; f0 < total_f && ok; f0 += G::PREFETCH) {
-#pragma unroll
-            for (int d = 0; d < G::PREFETCH; ++d) {
-                const int f = f0 + d;
-                if (f >= total_f || !ok) break;
-                const int slot = f % G::STAGES;
-                const uint32_t ph = static_cast<uint32_t>(f / G::STAGES) & 1u;
-                if (!mbar_wait(&empty[slot], ph ^ 1u, deadline)) { ok = false; break; }
-                uint8_t* stage = smem + slot * G::Q_BYTES;
-                if (lane == 0) {
-                    const int u = static_cast<int>(blockIdx.x) + (f / nst) * static_cast<int>(gridDim.x);
-                    const int st = f % nst;
-                    int grp, r0;
-                    unit_row0(u, grp, r0);
-                    const int row = static_cast<int>(static_cast<int64_t>(grp) * wrows + r0);
-                    mbar_arrive_expect_tx(&full[slot], G::Q_BYTES);
-#pragma unroll
-                    for (int m = 0; m < G::MAT; ++m)
-#pragma unroll
-                        for (int b = 0; b < NB; ++b)
-                            tma_load_2d(stage + (m * NB + b) * mxt::BOX_BYTES, &map_q, &full[slot],
-                                        (st * NB + b) * 128, row + m * p.I);
-                }
-                float* sc = reinterpret_cast<float*>(sc_ring + slot * G::SC_BYTES);
-#pragma unroll
-                for (int m = 0; m < G::NS; ++m) sc[lane + 32 * m] = e8m0_to_float(sreg[d][m]);
-                mbar_arrive(&full[slot]);
-                load_scales(f + G::PREFETCH, sreg[d]);
-            }
-        }
-        if (!ok) raise_error(p.err_flag, MOE_ERR_TIMEOUT);
-        return;
-    }
-
     // ---------------------------------------------------------------- consumers
     const int cw = warp - 1, g = lane >> 2, q = lane & 3;
     bool ok = true;
@@ -395,9 +325,8 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
         uint4 bv[G::BPW], bn[G::BPW];
         load_b(0, bv);
         // block scales of this lane's weight rows (g, g+8; KIND 0 also the up
-        // rows), loaded by the consumers one stage ahead when the producer does
-        // not stage them
-        constexpr int SR = KIND == 0 ? 4 : 2;
+        // rows), loaded one stage ahead like the activation fragments
+        constexpr int SR = G::SR;
         const uint8_t* srow[SR];
         bool sok[SR];
         {
@@ -410,7 +339,6 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
             }
         }
         auto load_s = [&](int st, uint32_t (&v)[G::BPW][SR]) {
-            if (!MOE_MX_CONSUMER_SCALES) return;
 #pragma unroll
             for (int i = 0; i < G::BPW; ++i) {
                 const int blk = st * G::BPS + cw * G::BPW + i;
@@ -428,7 +356,6 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
             load_s(st + 1, sn);
             if (ok && !mbar_wait(&full[slot], ph, deadline)) ok = false;
             const uint8_t* stage = smem + slot * G::Q_BYTES;
-            const float* sc = reinterpret_cast<const float*>(sc_ring + slot * G::SC_BYTES);
 #pragma unroll
             for (int i = 0; i < G::BPW; ++i) {
                 const int jj = cw * G::BPW + i;                  // block within the stage
@@ -442,25 +369,13 @@ __global__ void __launch_bounds__(mxt::THREADS, MOE_MX_MIN_BLOCKS) decode_mx_ker
                     const uint32_t v1 = *reinterpret_cast<const uint32_t*>(ux + (g + 8) * 128 + swz);
                     float tg[4] = {acc[0], acc[1], acc[2], acc[3]};
                     float tu[4] = {acc[4], acc[5], acc[6], acc[7]};
-                    if (MOE_MX_CONSUMER_SCALES) {
-                        mx_block(tg, w0, w1, bv[i], e8m0_to_float(sv[i][0]),
-                                 e8m0_to_float(sv[i][1]));
-                        mx_block(tu, v0, v1, bv[i], e8m0_to_float(sv[i][2]),
-                                 e8m0_to_float(sv[i][3]));
-                    } else {
-                        mx_block(tg, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
-                        mx_block(tu, v0, v1, bv[i], sc[(16 + g) * G::BPS + jj],
-                                 sc[(24 + g) * G::BPS + jj]);
-                    }
+                    mx_block(tg, w0, w1, bv[i], e8m0_to_float(sv[i][0]), e8m0_to_float(sv[i][1]));
+                    mx_block(tu, v0, v1, bv[i], e8m0_to_float(sv[i][2]), e8m0_to_float(sv[i][3]));
 #pragma unroll
                     for (int j = 0; j < 4; ++j) { acc[j] = tg[j]; acc[4 + j] = tu[j]; }
                 } else {
                     float t4[4] = {acc[0], acc[1], acc[2], acc[3]};
-                    if (MOE_MX_CONSUMER_SCALES)
-                        mx_block(t4, w0, w1, bv[i], e8m0_to_float(sv[i][0]),
-                                 e8m0_to_float(sv[i][SR - 1]));
-                    else
-                        mx_block(t4, w0, w1, bv[i], sc[g * G::BPS + jj], sc[(g + 8) * G::BPS + jj]);
+                    mx_block(t4, w0, w1, bv[i], e8m0_to_float(sv[i][0]), e8m0_to_float(sv[i][1]));
 #pragma unroll
                     for (int j = 0; j < 4; ++j) acc[j] = t4[j];
                 }
