@@ -56,3 +56,44 @@ def test_zipf_calibration_reaches_target():
     load = torch.bincount(sel.reshape(-1), minlength=cfg.E).double() / cfg.T
     q = torch.from_numpy(inp["zipf_target"])
     assert float((load - q).abs().max()) < 0.03
+
+
+def test_mxfp4_weights_are_seeded_and_shaped():
+    from sparse_mixture_experts_07_b200.inputs import MXFP4_SCALE_CODES, make_mxfp4_weights
+    cfg = MoEConfig("mx", T=2, H=128, I=96, E=3, k=1)
+    a = make_mxfp4_weights(cfg, seed=7)
+    b = make_mxfp4_weights(cfg, seed=7)
+    assert a["gate_up_q"].shape == (3, 192, 64) and a["gate_up_s"].shape == (3, 192, 4)
+    assert a["down_q"].shape == (3, 128, 48) and a["down_s"].shape == (3, 128, 3)
+    for key in a:
+        assert a[key].dtype == torch.uint8 and torch.equal(a[key], b[key])
+    scales = torch.cat([a["gate_up_s"].flatten(), a["down_s"].flatten()])
+    assert set(scales.tolist()) <= set(MXFP4_SCALE_CODES)
+    with pytest.raises(ValueError):
+        make_mxfp4_weights(MoEConfig("bad", T=1, H=136, I=96, E=2, k=1))
+
+
+def test_bench_rejects_mxfp4_outside_decode():
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--config", "mixtral",
+                        "--weights", "mxfp4"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 2 and "decode configuration" in r.stderr
+
+
+def test_decode_roofline_bytes():
+    import importlib.util
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    cfg = CONFIGS["phimoe_decode1"]
+    counts = np.zeros(cfg.E, dtype=np.int32)
+    counts[[3, 9]] = 1
+    act = 2 * cfg.T * cfg.H * 2 + 2 * cfg.T * cfg.k * cfg.H * 2 + cfg.E * cfg.H * 4
+    assert bench.bytes_decode(cfg, counts) == 2 * 3 * cfg.H * cfg.I * 2 + act
+    assert bench.bytes_decode(cfg, counts, mxfp4=True) == \
+        2 * 3 * cfg.H * cfg.I * (0.5 + 1 / 32) + act
