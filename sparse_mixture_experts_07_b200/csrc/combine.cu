@@ -64,8 +64,67 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_sl
     }
 }
 
+// bf16, H % 8 == 0: a persistent grid; each CTA walks its tokens t, t + grid,
+// ... and loads the slot indices of its next token while it sums the current
+// one, so the index round trip overlaps the row loads.  Same sum, same order.
+__global__ void __launch_bounds__(256) combine_bf16_pipelined_kernel(
+    const uint4* __restrict__ y_slots, const int32_t* __restrict__ inv, uint4* __restrict__ y,
+    int64_t n_tokens, int vec_per_row, int k, int S) {
+    const int64_t routed_rows = n_tokens * k;
+    const int nrows = k + S;
+    int64_t t = blockIdx.x;
+    // the threads < k fetch one slot index each for the next token
+    int32_t next_idx = (t < n_tokens && static_cast<int>(threadIdx.x) < k)
+                           ? inv[t * k + threadIdx.x] : 0;
+    __shared__ int64_t rows_sh[2][kMaxK + kMaxShared];
+    int buf = 0;
+    for (; t < n_tokens; t += gridDim.x) {
+        if (static_cast<int>(threadIdx.x) < k) rows_sh[buf][threadIdx.x] = next_idx;
+        if (static_cast<int>(threadIdx.x) < S)
+            rows_sh[buf][k + threadIdx.x] = routed_rows + threadIdx.x * n_tokens + t;
+        __syncthreads();
+        const int64_t tn = t + gridDim.x;
+        if (tn < n_tokens && static_cast<int>(threadIdx.x) < k) next_idx = inv[tn * k + threadIdx.x];
+        for (int v = threadIdx.x; v < vec_per_row; v += 256) {
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+            for (int j = 0; j < nrows; ++j) {
+                const uint4 u = y_slots[rows_sh[buf][j] * vec_per_row + v];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[2 * q] += bf16_to_f32(static_cast<uint16_t>(w[q] & 0xffffu));
+                    acc[2 * q + 1] += bf16_to_f32(static_cast<uint16_t>(w[q] >> 16));
+                }
+            }
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            y[t * vec_per_row + v] = o;
+        }
+        buf ^= 1;
+    }
+}
+
 cudaError_t launch_combine(const moe_shape& s, const void* y_slots, const int32_t* inv, void* y,
                            cudaStream_t st) {
+#ifndef MOE_COMBINE_PIPELINED
+#define MOE_COMBINE_PIPELINED 1
+#endif
+    if (MOE_COMBINE_PIPELINED && s.dtype == MOE_BF16) {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t cap = static_cast<int64_t>(sms) * 8;    // 8 CTAs of 256 threads per SM
+        const unsigned grid = static_cast<unsigned>(s.T < cap ? s.T : cap);
+        combine_bf16_pipelined_kernel<<<grid, 256, 0, st>>>(
+            static_cast<const uint4*>(y_slots), inv, static_cast<uint4*>(y), s.T, s.H / 8, s.k,
+            s.n_shared);
+        return cudaGetLastError();
+    }
     const unsigned grid = static_cast<unsigned>(s.T < 1048576 ? s.T : 1048576);
     if (s.dtype == MOE_BF16) {
         combine_kernel<__nv_bfloat16, 8><<<grid, 256, 0, st>>>(
