@@ -136,11 +136,15 @@ MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const float*
  * It returns MOE_ERR_UNSUPPORTED when the size above is 0 or a pointer is not
  * 16-byte aligned, and MOE_ERR_WORKSPACE when w_split_bytes is too small.
  *
- * moe_route_split computes exactly what moe_route computes, with the same
- * arguments plus `w_split` (the output of moe_router_split for this shape and
- * weight, or NULL).  For more than 256 tokens with bf16 x and E <= 64 it runs
- * the tensor-core router on w_split; its results are bit-identical to
- * moe_route's.  Otherwise, or when w_split is NULL, it is moe_route.
+ * moe_route_split computes what moe_route computes, with the same arguments
+ * plus `w_split` (the output of moe_router_split for this shape and weight,
+ * or NULL).  For more than 256 tokens with bf16 x and E <= 64 it runs the
+ * tensor-core router on w_split.  When the 128-token tiles alone would leave
+ * SMs idle, a cluster of up to 8 CTAs splits H between them; CTA c forms its
+ * partial logit (x.hi + x.mid) + x.lo over its slice and CTA 0 adds
+ * bias + p_0 + p_1 + ... in rank order.  That is a different float32
+ * summation order from moe_route's, within the same error bound; the result
+ * is deterministic.  Otherwise, or when w_split is NULL, it is moe_route.
  * A w_split that does not match w_router gives the routing of the weight it
  * was split from. */
 MOE_API moe_status moe_router_split_size(const moe_shape* shape, size_t* bytes);
