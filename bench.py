@@ -176,23 +176,65 @@ def bytes_decode(cfg, counts, mxfp4: bool = False) -> float:
         2 * cfg.T * (cfg.k + cfg.n_shared) * cfg.H * eb
 
 
+def cpu_oracle_rate_mxfp4(cfg, host_inp, mx_host, budget_s: float = 12.0,
+                          max_tokens: int = 4096):
+    """Oracle tokens/s of the MXFP4 block (numpy dequantisation of the selected
+    experts, then the float64 expert arithmetic) on a bounded token sample."""
+    import oracle
+    from oracle import mxfp4 as oracle_mx
+    oracle.build()
+    n = 1
+    rng = np.random.default_rng(1)
+    while True:
+        toks = rng.choice(cfg.T, size=min(n, cfg.T), replace=False)
+        t0 = time.perf_counter()
+        oracle_mx.moe_block_mxfp4(host_inp["x"], host_inp["w_router"], host_inp["router_bias"],
+                                  mx_host["gate_up_q"], mx_host["gate_up_s"], mx_host["down_q"],
+                                  mx_host["down_s"], k=cfg.k, routed_scale=cfg.routed_scale,
+                                  tokens=toks)
+        elapsed = time.perf_counter() - t0
+        if elapsed > budget_s / 4 or n >= min(cfg.T, max_tokens):
+            break
+        n *= 4
+    return len(toks) / elapsed, len(toks), elapsed, oracle.threads()
+
+
+def weights_label(args, cfg) -> str:
+    return "mxfp4 (E2M1 codes, E8M0 scales per 32)" if args.weights == "mxfp4" else cfg.dtype
+
+
 def run_reference(args, cfg, rank, world):
+    """The oracle arm: the CPU oracle, as it stands, timed on the host cores on
+    bounded token samples of the workload (rank 0 only; other ranks do no work)."""
     if rank != 0:
-        return
+        return None
     inp = make_inputs(cfg, seed=0, weights_device="cpu")
+    mx_host = None
+    if args.weights == "mxfp4":
+        from sparse_mixture_experts_07_b200.inputs import make_mxfp4_weights
+        mx_host = make_mxfp4_weights(cfg, seed=0, device="cpu")
+
+    def rate(budget, max_tokens):
+        if mx_host is not None:
+            return cpu_oracle_rate_mxfp4(cfg, inp, mx_host, budget_s=budget, max_tokens=max_tokens)
+        return cpu_oracle_rate(cfg, inp, budget_s=budget, max_tokens=max_tokens)
+
     # each step samples tokens for a bounded time, so that K steps stay within
     # about three minutes whatever K is
     step_budget = max(0.2, min(4.0, 180.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_oracle_rate(cfg, inp, budget_s=step_budget, max_tokens=16)
+        rate(step_budget, 16)
     rates, samples = [], []
+    cores = 1
     t_all = time.perf_counter()
     for _ in range(args.steps):
-        r, n, el, cores = cpu_oracle_rate(cfg, inp, budget_s=step_budget, max_tokens=256)
+        r, n, el, cores = rate(step_budget, 256)
         rates.append(r)
         samples.append(n)
     wall = time.perf_counter() - t_all
     value = statistics.median(rates)
+    what = "the MXFP4 block (numpy dequantisation of the selected experts, float64 expert " \
+           "math)" if mx_host is not None else "the block, float64"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.T / value,
@@ -200,17 +242,17 @@ def run_reference(args, cfg, rank, world):
         "data": "synthetic (seeded; shapes of the named model, random-init weights)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E,
                    "k": cfg.k, "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
-                   "routed_scale": cfg.routed_scale,
-                   "weights": "mxfp4 (E2M1 codes, E8M0 scales per 32)" if mx is not None
-                              else cfg.dtype, "storage": cfg.dtype},
+                   "routed_scale": cfg.routed_scale, "weights": weights_label(args, cfg),
+                   "storage": cfg.dtype},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"each step: the block for {samples[-1]} random tokens of the "
-                                   f"{cfg.T}-token batch (full routing of those tokens, all their "
-                                   f"experts), float64; rate extrapolated per token"},
+                         "sample": f"each step: {what} for {samples[-1] if samples else 0} "
+                                   f"random tokens of the {cfg.T}-token batch (full routing of "
+                                   f"those tokens, all their experts); rate per token"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
     }
     print(json.dumps(line), flush=True)
+    return line
 
 
 def count_launches(step_fn) -> int:
@@ -231,22 +273,137 @@ def count_launches(step_fn) -> int:
     return n
 
 
+def roofline_of(cfg, counts, fwd_ms, region_s, mxfp4, peaks, traffic=None) -> dict:
+    """Roofline of the dominant region (moe_forward) from its mean device time.
+
+    Decode batches (T*k <= 256) are HBM-bound: algorithmic bytes (bytes_decode)
+    per launch / time, against the measured HBM copy bandwidth.  Prefill is
+    tensor-bound: 2*T*(3kHI + 3 S Is H) flops per launch / time, against the
+    measured bf16 GEMM throughput (sustained when the timed region is long
+    enough to reach the power cap, else the burst figure)."""
+    if cfg.T * cfg.k <= 256:
+        algo = bytes_decode(cfg, counts, mxfp4=mxfp4)
+        achieved = algo / (fwd_ms / 1000.0) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "algorithmic_bytes": algo,
+                "kernel": "moe_forward_mxfp4 (f16 prep + MXFP4 expert FFN launches)"
+                          if mxfp4 else "moe_forward (expert FFN launches)",
+                "peak_kind": f"{peaks['source']} HBM copy"}
+    flops = 2.0 * cfg.T * (3 * cfg.k * cfg.H * cfg.I + 3 * cfg.n_shared * cfg.I_shared * cfg.H)
+    achieved = flops / (fwd_ms / 1000.0) / 1e12
+    # a timed region of back-to-back GEMMs longer than ~0.25 s runs into the
+    # power cap: compare with the sustained GEMM figure, else the burst one
+    long_run = region_s >= 0.25 and peaks["bf16_tflops_sustained"]
+    peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic,
+            "kernel": "moe_forward (gather + grouped GEMM gate_up/SwiGLU + grouped GEMM down)",
+            "peak_kind": f"{peaks['source']} bf16 {'sustained' if long_run else 'burst'}",
+            "frac_of_burst": achieved / peaks["bf16_tflops"]}
+
+
+class Workload:
+    """One configuration on the device: seeded inputs, the layer, its buffers."""
+
+    def __init__(self, cfg, weights: str, dev, seed: int):
+        import sparse_mixture_experts_07_b200 as moe
+        self.moe = moe
+        self.cfg = cfg
+        self.inp = make_inputs(cfg, seed=seed, weights_device=str(dev))
+        self.shape = moe.Shape.from_config(cfg)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.inp.items()}
+        self.mx = None
+        if weights == "mxfp4":
+            from sparse_mixture_experts_07_b200.inputs import make_mxfp4_weights
+            self.mx = make_mxfp4_weights(cfg, seed=seed, device=str(dev))
+            self.layer = moe.MoELayer(self.shape, d["w_router"], d["router_bias"], mxfp4=self.mx)
+        else:
+            self.layer = moe.MoELayer(self.shape, d["w_router"], d["router_bias"], d["gate_up"],
+                                      d["down"], d["sh_gate_up"], d["sh_down"])
+        self.x = d["x"]
+
+    def weight_bytes(self) -> int:
+        if self.mx is not None:
+            return sum(v.numel() for v in self.mx.values())
+        eb = 2 if self.cfg.dtype == "bf16" else 4
+        n = self.inp["gate_up"].numel() + self.inp["down"].numel()
+        if self.inp["sh_gate_up"] is not None:
+            n += self.inp["sh_gate_up"].numel() + self.inp["sh_down"].numel()
+        return n * eb
+
+    def step(self, stream, fwd_start=None, fwd_end=None):
+        """route -> permute -> forward -> combine, with events around the forward."""
+        moe, s, L = self.moe, self.shape, self.layer
+        b = L.buf
+        idx, w, _ = moe.route(s, self.x, L.w_router, L.router_bias, out=b, w_split=L.w_split,
+                              err_flag=L.err_flag, stream=stream)
+        moe.permute(s, idx, L.workspace, L.err_flag, out=b, stream=stream)
+        if fwd_start is not None:
+            fwd_start.record(stream)
+        if self.mx is not None:
+            moe.forward_mxfp4(s, self.x, b["offsets"], b["perm"], w, self.mx, L.workspace,
+                              L.err_flag, y_slots=b["y_slots"], stream=stream)
+        else:
+            moe.forward(s, self.x, b["offsets"], b["perm"], w, L.gate_up, L.down, L.sh_gate_up,
+                        L.sh_down, L.workspace, L.err_flag, y_slots=b["y_slots"], stream=stream)
+        if fwd_end is not None:
+            fwd_end.record(stream)
+        moe.combine(s, b["y_slots"], b["inv"], y=b["y"], stream=stream)
+
+
+# Secondary workloads timed after the headline one in a default run (1 GPU):
+# the decode batches (the HBM half of the metric) and the other prefill shapes.
+EXTRA_WORKLOADS = [
+    ("phimoe_decode1", "bf16"), ("phimoe_decode8", "bf16"), ("phimoe_decode64", "bf16"),
+    ("phimoe_decode1", "mxfp4"), ("phimoe_decode8", "mxfp4"), ("phimoe_decode64", "mxfp4"),
+    ("phimoe_prefill", "bf16"), ("gptoss", "bf16"), ("dsv3", "bf16"),
+]
+
+
+def measure_extra(name, weights, dev, steps, peaks, flush) -> dict:
+    """Device time of `steps` steps of one workload, each step timed on its own
+    with the L2 flushed in between when the step's weights would fit in L2."""
+    cfg = CONFIGS[name]
+    w = Workload(cfg, weights, dev, seed=0)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        w.step(stream)
+    torch.cuda.synchronize()
+    assert w.layer.device_error() == 0, f"device error flag set ({name})"
+    need_flush = w.weight_bytes() < 4 * L2_BYTES
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        if need_flush:
+            flush.zero_()
+        e0, e1, f0, f1 = ev[i]
+        e0.record(stream)
+        w.step(stream, f0, f1)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    assert w.layer.device_error() == 0, f"device error flag set ({name})"
+    step_ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    fwd_ms = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
+    counts = w.layer.buf["counts"].cpu().numpy()
+    roof = roofline_of(cfg, counts, fwd_ms, 0.0, w.mx is not None, peaks)
+    out = {"workload": name, "weights": weights, "T": cfg.T, "steps": steps,
+           "ms_per_step": step_ms, "tokens_per_s": cfg.T / (step_ms / 1000.0),
+           "forward_ms": fwd_ms, "roofline": {k: roof[k] for k in (
+               "bound", "achieved", "peak", "unit", "frac", "peak_kind")},
+           "l2": "L2 flushed before every step (256 MB write)" if need_flush
+                 else f"weights {w.weight_bytes() / 1e9:.2f} GB > L2, streamed every step",
+           "active_experts": int((counts > 0).sum())}
+    del w
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_cuda(args, cfg, rank, local, world):
     import sparse_mixture_experts_07_b200 as moe
 
     dev = torch.device("cuda", local)
-    inp = make_inputs(cfg, seed=rank, weights_device=str(dev))
-    shape = moe.Shape.from_config(cfg)
-    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    mx = None
-    if args.weights == "mxfp4":
-        from sparse_mixture_experts_07_b200.inputs import make_mxfp4_weights
-        mx = make_mxfp4_weights(cfg, seed=rank, device=str(dev))
-        layer = moe.MoELayer(shape, d["w_router"], d["router_bias"], mxfp4=mx)
-    else:
-        layer = moe.MoELayer(shape, d["w_router"], d["router_bias"], d["gate_up"], d["down"],
-                             d["sh_gate_up"], d["sh_down"])
-    x = d["x"]
+    wl = Workload(cfg, args.weights, dev, seed=rank)
+    layer, x, mx, shape = wl.layer, wl.x, wl.mx, wl.shape
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -269,20 +426,7 @@ def run_cuda(args, cfg, rank, local, world):
     with ClockSampler(local) as clk:
         s0.record(stream)
         for i in range(args.steps):
-            idx, w, _ = moe.route(shape, x, layer.w_router, layer.router_bias, out=b,
-                                  w_split=layer.w_split,
-                                  err_flag=layer.err_flag)
-            moe.permute(shape, idx, layer.workspace, layer.err_flag, out=b)
-            fwd_start[i].record(stream)
-            if mx is not None:
-                moe.forward_mxfp4(shape, x, b["offsets"], b["perm"], w, mx, layer.workspace,
-                                  layer.err_flag, y_slots=b["y_slots"])
-            else:
-                moe.forward(shape, x, b["offsets"], b["perm"], w, layer.gate_up, layer.down,
-                            layer.sh_gate_up, layer.sh_down, layer.workspace, layer.err_flag,
-                            y_slots=b["y_slots"])
-            fwd_end[i].record(stream)
-            moe.combine(shape, b["y_slots"], b["inv"], y=b["y"])
+            wl.step(stream, fwd_start[i], fwd_end[i])
         s1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -346,38 +490,15 @@ def run_cuda(args, cfg, rank, local, world):
     assert layer.device_error() == 0, "device error flag set"
 
     peaks = measured_peaks()
-    decode = cfg.T * cfg.k <= 256
     tr = TRAFFIC.get(cfg.name)
     traffic = None
-    if tr:
+    if tr and mx is None:
         src = os.path.join(ROOT, "sparse_mixture_experts_07_b200", "csrc", tr["file"])
         if os.path.exists(src) and tr.get("sha") == src_sha(src):
             traffic = tr["bytes"]
-    if decode:
-        algo = bytes_decode(cfg, counts, mxfp4=mx is not None)
-        achieved = algo / (fwd_ms / 1000.0) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "moe_forward_mxfp4 (f16 prep + MXFP4 expert FFN launches)"
-                          if mx is not None else "moe_forward (expert FFN launches)",
-                "peak_kind": f"{peaks['source']} HBM copy"}
-    else:
-        flops = 2.0 * cfg.T * (3 * cfg.k * cfg.H * cfg.I + 3 * cfg.n_shared * cfg.I_shared * cfg.H)
-        achieved = flops / (fwd_ms / 1000.0) / 1e12
-        # a timed region of back-to-back GEMMs longer than ~0.25 s runs into the
-        # power cap: compare with the sustained GEMM figure, else the burst one
-        long_run = ms_total / 1000.0 >= 0.25 and peaks["bf16_tflops_sustained"]
-        peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "kernel": "moe_forward (gather + grouped GEMM gate_up/SwiGLU + grouped GEMM down)",
-                "peak_kind": f"{peaks['source']} bf16 {'sustained' if long_run else 'burst'}",
-                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    roof = roofline_of(cfg, counts, fwd_ms, ms_total / 1000.0, mx is not None, peaks, traffic)
+    roof.pop("algorithmic_bytes", None)
 
-    if mx is not None:
-        weight_bytes = sum(v.numel() for v in mx.values())
-    else:
-        weight_bytes = (inp["gate_up"].numel() + inp["down"].numel()) * eb
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
@@ -386,12 +507,10 @@ def run_cuda(args, cfg, rank, local, world):
         "data": "synthetic (seeded; shapes of the named model, random-init weights)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E,
                    "k": cfg.k, "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
-                   "routed_scale": cfg.routed_scale,
-                   "weights": "mxfp4 (E2M1 codes, E8M0 scales per 32)" if mx is not None
-                              else cfg.dtype,
+                   "routed_scale": cfg.routed_scale, "weights": weights_label(args, cfg),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (expert weights "
-                         f"{weight_bytes / 1e9:.2f} GB streamed every step)"},
+                         f"{wl.weight_bytes() / 1e9:.2f} GB streamed every step)"},
         "tflops": 2.0 * cfg.T * (cfg.H * cfg.E + 3 * cfg.k * cfg.H * cfg.I +
                                  3 * cfg.n_shared * cfg.I_shared * cfg.H) * args.steps * world /
                   (ms_total / 1000.0) / 1e12,
@@ -403,31 +522,38 @@ def run_cuda(args, cfg, rank, local, world):
         "expert_counts": counts.tolist(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and mx is not None:
-        # the oracle's MXFP4 block on the whole (decode) batch: dequantise the
-        # selected experts, then the float64 expert math
-        import oracle
-        from oracle import mxfp4 as oracle_mx
-        host = host_inputs(inp)
+        host = host_inputs(wl.inp)
         hm = {k: v.cpu() for k, v in mx.items()}
-        t0 = time.perf_counter()
-        oracle_mx.moe_block_mxfp4(host["x"], host["w_router"], host["router_bias"],
-                                  hm["gate_up_q"], hm["gate_up_s"], hm["down_q"], hm["down_s"],
-                                  k=cfg.k, routed_scale=cfg.routed_scale)
-        el = time.perf_counter() - t0
+        r, n, el, cores = cpu_oracle_rate_mxfp4(cfg, host, hm)
         line["cpu_baseline"] = {
-            "value": cfg.T / el, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"the MXFP4 block for all {cfg.T} tokens ({el:.1f} s: numpy dequantisation "
-                      "of the selected experts, then float64 expert math)"}
+            "value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"the MXFP4 block for {n} of the {cfg.T} tokens ({el:.1f} s: numpy "
+                      "dequantisation of the selected experts, then float64 expert math)"}
     elif rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = host_inputs(inp)
+        host = host_inputs(wl.inp)
         r, n, el, cores = cpu_oracle_rate(cfg, host)
         line["cpu_baseline"] = {
             "value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"the block for {n} random tokens of the {cfg.T}-token batch "
                       f"({el:.1f} s, float64, OpenMP over tokens); rate per token"}
+    del layer, wl, x_host, y_host, x_dev, y_dev
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads (1 GPU only): decode batches and prefill shapes,
+    # each with the roofline fraction of its forward
+    if world == 1 and not args.no_extra:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        extra = []
+        with ClockSampler(local) as clk2:
+            for name, weights in EXTRA_WORKLOADS:
+                if name == cfg.name and weights == args.weights:
+                    continue
+                extra.append(measure_extra(name, weights, dev, max(10, min(args.steps, 50)),
+                                           peaks, flush))
+        line["workloads"] = extra
+        line["workloads_clocks"] = clk2.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del layer
 
 
 def main():
@@ -438,12 +564,14 @@ def main():
     ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the headline workload (skip the decode and prefill lines)")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"],
-                    help="expert weight format; mxfp4 runs the decode path (T <= 8)")
+                    help="expert weight format; mxfp4 runs the decode path (T <= 64)")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
-    if args.weights == "mxfp4" and not (cfg.T <= 8 and cfg.dtype == "bf16" and cfg.n_shared == 0):
-        ap.error("--weights mxfp4 needs a bf16 decode configuration (T <= 8, no shared experts)")
+    if args.weights == "mxfp4" and not (cfg.T <= 64 and cfg.dtype == "bf16" and cfg.n_shared == 0):
+        ap.error("--weights mxfp4 needs a bf16 decode configuration (T <= 64, no shared experts)")
     rank, local, world = dist_setup()
     try:
         if args.impl == "reference":
