@@ -314,3 +314,201 @@ def test_configs_follow_page_shapes():
     assert CONFIGS["mixtral"].k == g["mixtral.num_experts_per_tok"]
     from sparse_mixture_experts_07_b200.inputs import INIT_STD
     assert INIT_STD == g["phimoe.initializer_range"]
+
+
+# ------------------------------------------------- expert-parallel partials
+@pytest.mark.parametrize("bounds", [(0, 2, 4, 6), (0, 1, 6), (0, 3, 3, 6), (0, 6)])
+def test_expert_partials_over_a_partition_sum_to_the_block(bounds):
+    """The ranks' partials (each its range of experts, shared experts on the
+    first rank only) sum to the whole block; a rank without experts and
+    without the shared experts contributes zero."""
+    inp = _rand_inputs(10, 12, 8, 6, S=2, Is=5, seed=11, bias=True)
+    y, _, _ = oracle.moe_block(inp, k=3, routed_scale=2.5)
+    parts = [oracle.moe_block_experts(inp, k=3, routed_scale=2.5, e_begin=a, e_end=b,
+                                      with_shared=(r == 0))
+             for r, (a, b) in enumerate(zip(bounds[:-1], bounds[1:]))]
+    assert _rel_l2(sum(parts), y) < 1e-13
+    for (a, b), part in zip(zip(bounds[:-1], bounds[1:]), parts):
+        if a == b and part is not parts[0]:
+            assert not part.any()
+
+
+def test_expert_partial_of_one_expert_is_its_weighted_output():
+    inp = _rand_inputs(6, 8, 5, 4, seed=12, bias=True)
+    lg = oracle.router(inp["x"], inp["w_router"], inp["router_bias"])
+    idx, w = oracle.topk_softmax(lg, 2)
+    part = oracle.moe_block_experts(inp, k=2, routed_scale=1.0, e_begin=1, e_end=2)
+    for t in range(6):
+        ref = np.zeros(8)
+        for j in range(2):
+            if idx[t, j] == 1:
+                ref = w[t, j] * oracle.expert(inp["gate_up"][1], inp["down"][1],
+                                              inp["x"][t].double().numpy())
+        assert np.allclose(part[t], ref, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------- DeepSeek-V3 (noaux_tc) routing
+def _sigmoid(v):
+    return 1.0 / (1.0 + math.exp(-v))
+
+
+def test_noaux_without_groups_or_bias_is_topk_of_the_logits():
+    """One group and no bias: sigmoid is increasing, so the selection is the
+    plain top-k of the logits, and the weights are the selected sigmoids
+    normalised."""
+    rng = np.random.default_rng(21)
+    lg = rng.normal(size=(40, 16))
+    idx, w = oracle.route_noaux_tc(lg, None, 4, 1, 1)
+    idx_ref, _ = oracle.topk_softmax(lg, 4)
+    assert np.array_equal(idx, idx_ref)
+    for t in range(40):
+        s = np.array([_sigmoid(lg[t, e]) for e in idx[t]])
+        assert np.allclose(w[t], s / s.sum(), rtol=1e-14, atol=0)
+    assert np.allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+
+
+def test_noaux_bias_moves_the_selection_but_not_the_weights():
+    lg = np.array([[2.0, 1.0, 0.0, -1.0]])
+    bias = np.array([0.0, 0.0, 0.0, 5.0], dtype=np.float32)
+    idx, w = oracle.route_noaux_tc(lg, bias, 2, 1, 1)
+    assert idx.tolist() == [[3, 0]]            # 5 + sigmoid(-1) first, then sigmoid(2)
+    s3, s0 = _sigmoid(-1.0), _sigmoid(2.0)
+    assert np.allclose(w[0], [s3 / (s3 + s0), s0 / (s3 + s0)], rtol=1e-14, atol=0)
+
+
+def test_noaux_hand_worked_group_limited_selection():
+    """E=8 in 4 groups of 2, keep 2 groups, k=3.  Affinities (sigmoid of the
+    logits) 0.953 0.047 | 0.881 0.870 | 0.924 0.018 | 0.500 0.525; group scores
+    (sums) 1.000, 1.751, 0.942, 1.025, so groups 1 and 3 are kept and the two
+    largest affinities overall (experts 0 and 4) are excluded."""
+    lg = np.array([[3.0, -3.0, 2.0, 1.9, 2.5, -4.0, 0.0, 0.1]])
+    idx, w = oracle.route_noaux_tc(lg, None, 3, 4, 2)
+    assert idx.tolist() == [[2, 3, 7]]
+    s = np.array([_sigmoid(2.0), _sigmoid(1.9), _sigmoid(0.1)])
+    assert np.allclose(w[0], s / s.sum(), rtol=1e-14, atol=0)
+    # keeping every group removes the restriction: the plain top-3
+    idx_all, _ = oracle.route_noaux_tc(lg, None, 3, 4, 4)
+    assert idx_all.tolist() == [[0, 4, 2]]
+
+
+def test_noaux_keeping_all_groups_equals_one_group():
+    rng = np.random.default_rng(22)
+    lg = rng.normal(size=(30, 24))
+    bias = rng.normal(scale=0.3, size=24).astype(np.float32)
+    a = oracle.route_noaux_tc(lg, bias, 5, 1, 1)
+    b = oracle.route_noaux_tc(lg, bias, 5, 6, 6)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_noaux_selected_experts_lie_in_the_best_groups():
+    """With 8 groups of 8 and 4 kept, every selected expert's group is among
+    the 4 groups with the largest two-expert sums; permuting whole groups
+    permutes the selection with them."""
+    rng = np.random.default_rng(23)
+    E, G, kg, k = 64, 8, 4, 6
+    lg = rng.normal(size=(50, E))
+    bias = rng.normal(scale=0.2, size=E).astype(np.float32)
+    idx, _ = oracle.route_noaux_tc(lg, bias, k, G, kg)
+    c = 1.0 / (1.0 + np.exp(-lg)) + bias.astype(np.float64)
+    gs = np.sort(c.reshape(50, G, E // G), axis=2)[:, :, -2:].sum(axis=2)
+    kept = np.argsort(-gs, axis=1)[:, :kg]
+    for t in range(50):
+        assert set((idx[t] // (E // G)).tolist()) <= set(kept[t].tolist())
+    order = rng.permutation(G)
+    cols = np.concatenate([np.arange(g * 8, g * 8 + 8) for g in order])
+    idx2, _ = oracle.route_noaux_tc(lg[:, cols], bias[cols], k, G, kg)
+    assert np.array_equal(cols[idx2], idx)
+
+
+def test_routed_block_with_softmax_routing_is_the_block():
+    inp = _rand_inputs(9, 12, 8, 6, S=1, Is=5, seed=24, bias=True)
+    y, idx, w = oracle.moe_block(inp, k=2, routed_scale=2.5)
+    y2 = oracle.moe_block_routed(inp, idx, w, routed_scale=2.5)
+    assert _rel_l2(y2, y) < 1e-14
+    toks = [8, 0, 3]
+    y3 = oracle.moe_block_routed(inp, idx[toks], w[toks], routed_scale=2.5, tokens=toks)
+    assert _rel_l2(y3, y[toks]) < 1e-14
+
+
+# ------------------------------------------------------------ backward pass
+def _loss(inp, k, dy, scale):
+    y, _, _ = oracle.moe_block(inp, k=k, routed_scale=scale)
+    return float((y * dy).sum())
+
+
+def _fd_check(inp, name, k, dy, scale, grad, n_pick, rng, delta=2.0 ** -12):
+    """Central differences of L = <dy, y> against the analytic gradient, on
+    n_pick random entries of the float32 tensor inp[name]; each perturbation
+    is a power of two, exact in float32, so the difference quotient is
+    float64-accurate up to O(delta^2)."""
+    t = inp[name]
+    flat = t.view(-1)
+    for i in rng.choice(flat.numel(), size=min(n_pick, flat.numel()), replace=False):
+        old = float(flat[i])
+        flat[i] = old + delta
+        lp = _loss(inp, k, dy, scale)
+        flat[i] = old - delta
+        lm = _loss(inp, k, dy, scale)
+        flat[i] = old
+        fd = (lp - lm) / (2 * delta)
+        g = float(grad.reshape(-1)[i])
+        assert abs(fd - g) <= 1e-6 * max(1.0, abs(g)) + 1e-9, (name, int(i), fd, g)
+
+
+@pytest.mark.parametrize("S", [0, 2])
+def test_backward_matches_finite_differences(S):
+    """Every gradient the oracle's backward returns (x, both expert weights,
+    router weight and bias, shared experts) agrees with central finite
+    differences of its own forward: an independent check of the chain rule."""
+    inp = _rand_inputs(6, 8, 5, 4, S=S, Is=3, seed=31, bias=True)
+    scale = 2.5 if S else 1.0
+    rng = np.random.default_rng(31)
+    dy = rng.normal(size=(6, 8))
+    gr = oracle.moe_backward(inp, 2, dy, routed_scale=scale)
+    names = ["x", "gate_up", "down", "w_router", "router_bias"]
+    if S:
+        names += ["sh_gate_up", "sh_down"]
+    for name in names:
+        _fd_check(inp, name, 2, dy, scale, gr[name], 24, rng)
+
+
+def test_backward_routing_weight_and_logit_gradients():
+    """dw_j = s <dy, f_j> (each expert's output read back from the block with
+    a one-hot weight) and dl is the softmax Jacobian over the selected k
+    applied to dw: zero off the selection, summing to zero per token."""
+    inp = _rand_inputs(5, 8, 6, 5, seed=32, bias=True)
+    rng = np.random.default_rng(32)
+    dy = rng.normal(size=(5, 8))
+    gr = oracle.moe_backward(inp, 3, dy, routed_scale=2.0)
+    y, idx, w = oracle.moe_block(inp, k=3, routed_scale=2.0)
+    for t in range(5):
+        xv = inp["x"][t].double().numpy()
+        for j in range(3):
+            f = oracle.expert(inp["gate_up"][idx[t, j]], inp["down"][idx[t, j]], xv)
+            assert np.isclose(gr["dw"][t, j], 2.0 * float(dy[t] @ f), rtol=1e-12, atol=1e-14)
+        off = np.setdiff1d(np.arange(5), idx[t])
+        assert np.all(gr["dl"][t, off] == 0.0)
+        assert abs(gr["dl"][t].sum()) < 1e-14
+    assert np.allclose(gr["router_bias"], gr["dl"].sum(axis=0), rtol=1e-13, atol=1e-15)
+
+
+def test_aux_loss_closed_forms_and_finite_differences():
+    T, E, k = 12, 6, 2
+    rng = np.random.default_rng(33)
+    # uniform router: p = 1/E, so the loss is coef * k and dl = coef/T (f - k/E)
+    lg = np.zeros((T, E))
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    loss, dl = oracle.aux_loss(lg, idx, E, coef=0.01)
+    f = np.bincount(idx.reshape(-1), minlength=E) / T
+    assert np.isclose(loss, 0.01 * k, rtol=1e-14)
+    assert np.allclose(dl, 0.01 / T * (f - k / E)[None, :], rtol=1e-13, atol=1e-17)
+    # random logits: central differences (the dispatch counts held fixed)
+    lg = rng.normal(size=(T, E))
+    loss, dl = oracle.aux_loss(lg, idx, E, coef=0.01)
+    for t, e in [(0, 0), (3, 5), (11, 2), (7, 1)]:
+        d = 1e-6
+        lp, lm = lg.copy(), lg.copy()
+        lp[t, e] += d
+        lm[t, e] -= d
+        fd = (oracle.aux_loss(lp, idx, E, 0.01)[0] - oracle.aux_loss(lm, idx, E, 0.01)[0]) / (2 * d)
+        assert abs(fd - dl[t, e]) <= 1e-9
