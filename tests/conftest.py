@@ -19,3 +19,18 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With PARITY_RECORD=<path>, write the errors the parity tests measured."""
+    path = os.environ.get("PARITY_RECORD")
+    if not path:
+        return
+    try:
+        import json
+
+        import parity_util
+        with open(path, "w") as f:
+            json.dump(parity_util.records(), f, indent=1, sort_keys=True)
+    except Exception:       # the record is a by-product; never fail the run on it
+        pass

@@ -97,3 +97,27 @@ def test_decode_roofline_bytes():
     assert bench.bytes_decode(cfg, counts) == 2 * 3 * cfg.H * cfg.I * 2 + act
     assert bench.bytes_decode(cfg, counts, mxfp4=True) == \
         2 * 3 * cfg.H * cfg.I * (0.5 + 1 / 32) + act
+
+
+def test_noaux_inputs_have_clear_selection_gaps():
+    """For DeepSeek-V3 routing the generator rejects near ties in the space the
+    selection is taken in: sigmoid(logit) + bias, with group-limited top-k."""
+    import oracle
+    from sparse_mixture_experts_07_b200.inputs import GAP
+    cfg = MoEConfig("nx_gen", T=400, H=128, I=64, E=32, k=4, zipf_s=1.0, routing="noaux_tc",
+                    n_group=4, topk_group=2)
+    inp = make_inputs(cfg, seed=3)
+    lg = oracle.router(inp["x"], inp["w_router"], None)
+    b = inp["router_bias"].numpy().astype(np.float64)
+    c = 1.0 / (1.0 + np.exp(-lg)) + b
+    gsize = cfg.E // cfg.n_group
+    gs = np.sort(c.reshape(cfg.T, cfg.n_group, gsize), axis=2)[:, :, -2:].sum(axis=2)
+    gsorted = -np.sort(-gs, axis=1)
+    assert (gsorted[:, cfg.topk_group - 1] - gsorted[:, cfg.topk_group] > GAP).all()
+    idx, _ = oracle.route_noaux_tc(lg, inp["router_bias"], cfg.k, cfg.n_group, cfg.topk_group)
+    kept = np.argsort(-gs, axis=1)[:, :cfg.topk_group]
+    for t in range(cfg.T):
+        allowed = np.concatenate([np.arange(g * gsize, (g + 1) * gsize) for g in kept[t]])
+        top = np.sort(c[t, allowed])[::-1][:cfg.k + 1]
+        assert (np.diff(-top) > GAP).all()
+        assert set(idx[t].tolist()) == set(allowed[np.argsort(-c[t, allowed])[:cfg.k]].tolist())

@@ -6,7 +6,8 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import (check_outputs, check_routing, run_gpu, sample_tokens, to_device)
+from parity_util import (check_outputs, check_routing, run_gpu, stratified_tokens,
+                         to_device)
 from sparse_mixture_experts_07_b200.inputs import CONFIGS, MoEConfig, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -112,18 +113,32 @@ def test_bad_expert_index_sets_error_flag(cuda_ok):
 FULL = ["mixtral", "phimoe_prefill", "gptoss", "dsv3", "phimoe_decode1", "phimoe_decode8",
         "phimoe_decode64"]
 
+# Tokens whose outputs are checked against the oracle at full size: every
+# routed expert's first row, the first and last row of its last 128-row tile
+# and two more of its rows, then random tokens up to this many (about 15-25 s
+# of oracle time each on 16 host cores).
+FULL_SAMPLE = {"mixtral": 768, "phimoe_prefill": 1024, "gptoss": 2048, "dsv3": 2048}
+
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_sampled(cuda_ok, name):
-    """Full-size configurations: routing for every token, the plan's
-    invariants, and the outputs of a sample of tokens against the oracle."""
+    """Full-size configurations: routing for every token, the plan bit-exact
+    against the oracle's, and the outputs of a stratified sample of tokens
+    (all tokens of the decode batches) against the oracle, over the sample
+    and row by row."""
     cfg = CONFIGS[name]
     inp = make_inputs(cfg, seed=0, weights_device="cuda")
     res = run_gpu(cfg, to_device(inp))
     assert res["err"] == 0
     host = {key: (v.cpu() if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
-    toks = sample_tokens(cfg.T, 24 if cfg.T > 64 else cfg.T)
-    check_routing(cfg, host, res)
+    o_idx, _, o_offsets, o_perm = check_routing(cfg, host, res)
+    if cfg.T <= 64:
+        toks = np.arange(cfg.T)
+    else:
+        toks = stratified_tokens(o_idx, o_offsets, o_perm, FULL_SAMPLE[name])
+        # every routed expert with slots has at least one checked row
+        hit = np.unique(o_idx[toks].reshape(-1))
+        assert np.array_equal(hit, np.nonzero(np.diff(o_offsets))[0])
     check_outputs(cfg, host, res, tokens=toks)
 
 

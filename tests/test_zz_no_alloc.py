@@ -5,9 +5,12 @@ owns every allocation and passes in only inputs and outputs; a latency-bound
 path where a cudaMalloc could synchronise the device).  For them the library
 keeps the plan's scratch in its own static device memory.  This file checks
 that entry point, called through the C ABI, against moe_permute on two calls
-in a row (a large plan, then a smaller one that reuses the array left dirty by
-the first).  It sorts last so that a failure here stops a -x run only after
-every other test has run.
+in a row.  Both plans are above 65536 slots, so both take the three-launch
+path that uses the static array: the first (120000 slots, 59 blocks x 64
+experts) fills 3776 entries of it, the second (72000 slots, 36 blocks x 32
+experts) reuses a prefix of the array that the first left dirty.  It sorts
+last so that a failure here stops a -x run only after every other test has
+run.
 """
 import ctypes
 
@@ -42,7 +45,8 @@ def test_noalloc_permute_matches_workspace_permute(cuda_ok):
     lib = moe.load_library()
     f = _noalloc(lib)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for T, E, k, seed in ((20000, 64, 6, 1), (777, 8, 2, 2)):
+    for T, E, k, seed in ((20000, 64, 6, 1), (12000, 32, 6, 2)):
+        assert T * k > 65536    # the path that uses the static array
         shape = moe.Shape(T=T, H=128, I=128, E=E, k=k)
         idx = _random_topk(T, E, k, seed)
         ws = moe.alloc_workspace(shape)
