@@ -398,6 +398,64 @@ def measure_extra(name, weights, dev, steps, peaks, flush) -> dict:
     return out
 
 
+def measure_train(name, dev, steps, peaks) -> dict:
+    """Device time of a training step of the layer: route, plan, the training
+    forward (which keeps g, u, h and the gathered x rows), the combine, and
+    the backward pass for a fixed upstream gradient.  The roofline counts the
+    expert GEMMs: 6 T k H I flops forward and twice that backward (plus the
+    shared experts)."""
+    import sparse_mixture_experts_07_b200 as moe
+    cfg = CONFIGS[name]
+    w = Workload(cfg, "bf16", dev, seed=0)
+    L, s, x = w.layer, w.shape, w.x
+    b = L.buf
+    state = torch.empty(moe.train_state_size(s), dtype=torch.uint8, device=dev)
+    bws = torch.empty(moe.backward_workspace_size(s), dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev).manual_seed(3)
+    dy = torch.randn(cfg.T, cfg.H, generator=g, device=dev).to(torch.bfloat16)
+    logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(f0=None, f1=None):
+        idx, wt, _ = moe.route(s, x, L.w_router, L.router_bias, out=b, w_split=L.w_split,
+                               err_flag=L.err_flag, stream=stream)
+        moe.permute(s, idx, L.workspace, L.err_flag, out=b, stream=stream)
+        if f0 is not None:
+            f0.record(stream)
+        moe.forward_train(s, x, b["offsets"], b["perm"], wt, L.gate_up, L.down, L.sh_gate_up,
+                          L.sh_down, L.workspace, state, L.err_flag, y_slots=b["y_slots"],
+                          stream=stream)
+        moe.combine(s, b["y_slots"], b["inv"], y=b["y"], stream=stream)
+        moe.backward(s, x, L.w_router, idx, wt, b["counts"], b["offsets"], b["perm"], b["inv"],
+                     L.gate_up, L.down, L.sh_gate_up, L.sh_down, state, dy, bws, L.err_flag,
+                     logits=logits, aux_coef=0.0, stream=stream)
+        if f1 is not None:
+            f1.record(stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    assert L.device_error() == 0, f"device error flag set (training {name})"
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for i in range(steps):
+        step(ev[i][0], ev[i][1])
+    torch.cuda.synchronize()
+    assert L.device_error() == 0, f"device error flag set (training {name})"
+    ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    fwd_flops = 2.0 * cfg.T * (3 * cfg.k * cfg.H * cfg.I + 3 * cfg.n_shared * cfg.I_shared * cfg.H)
+    achieved = 3.0 * fwd_flops / (ms / 1000.0) / 1e12
+    out = {"workload": name, "weights": "bf16", "kind": "training step (forward + backward)",
+           "T": cfg.T, "steps": steps, "train_ms": ms, "tokens_per_s": cfg.T / (ms / 1000.0),
+           "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                        "peak_kind": f"{peaks['source']} bf16 burst",
+                        "region": "training forward + backward of the expert FFNs "
+                                  "(flops of the six grouped GEMMs)"}}
+    del w, state, bws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_cuda(args, cfg, rank, local, world):
     import sparse_mixture_experts_07_b200 as moe
 
@@ -550,6 +608,8 @@ def run_cuda(args, cfg, rank, local, world):
                     continue
                 extra.append(measure_extra(name, weights, dev, max(10, min(args.steps, 50)),
                                            peaks, flush))
+            if not args.no_train:
+                extra.append(measure_train("mixtral", dev, max(5, min(args.steps, 20)), peaks))
         line["workloads"] = extra
         line["workloads_clocks"] = clk2.summary()
     if rank == 0:
@@ -566,6 +626,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="time only the headline workload (skip the decode and prefill lines)")
+    ap.add_argument("--no-train", action="store_true",
+                    help="skip the training-step line among the extra workloads")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"],
                     help="expert weight format; mxfp4 runs the decode path (T <= 64)")
     args = ap.parse_args()

@@ -155,6 +155,33 @@ MOE_API moe_status moe_route_split(const moe_shape* shape, const void* x, const 
                                    int32_t* topk_idx, float* topk_w, int32_t* err_flag,
                                    void* stream);
 
+/* DeepSeek-V3 routing, "noaux_tc" (named as the top-k method of the
+ * DeepSeek-V3-derived Instella-MoE, Instella-MoE walk-through, "config at a
+ * glance"; the pages do not define it, and this follows the DeepSeek-V3
+ * technical report, section 2.1):
+ *   s_e = sigmoid(l_e)  with l = x Wr^T (no bias in the logits)
+ *   c_e = s_e + score_bias[e]          the bias steers the selection only
+ *   experts form n_group contiguous groups of E / n_group; a group scores the
+ *   float32 sum of its two largest c_e; the topk_group best groups are kept
+ *   (ties to the lower group index); the k largest c_e among the kept groups
+ *   are selected in descending order (ties to the lower expert index);
+ *   topk_w[t, j] = s_(idx_j) / sum_i s_(idx_i)   (sums to 1; the routed
+ *   scale of the shape multiplies the routed sum later, in moe_forward).
+ * Arguments as moe_route_split, plus
+ *   n_group, topk_group  1 <= n_group <= 32, E % n_group == 0,
+ *                        1 <= topk_group <= n_group,
+ *                        k <= topk_group * E / n_group (else INVALID_ARG)
+ *   score_bias [E]       float32 selection bias, or NULL
+ *   logits     [T, E]    float32, REQUIRED: receives the bias-free logits,
+ *                        which the selection kernel then reads.
+ * Two launches: the router (moe_route_split with no bias), then one warp per
+ * token for the selection. */
+MOE_API moe_status moe_route_noaux_tc(const moe_shape* shape, int32_t n_group,
+                                      int32_t topk_group, const void* x, const float* w_router,
+                                      const void* w_split, const float* score_bias,
+                                      float* logits, int32_t* topk_idx, float* topk_w,
+                                      int32_t* err_flag, void* stream);
+
 /* Dropless dispatch plan ("Mixture of Experts in Transformers", grouped_mm
  * backend: sort and group tokens by expert id).  Slot q = t*k + j.
  *   topk_idx  [T, k]  int32 input
@@ -176,15 +203,19 @@ MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, 
  * its input and output buffers, or a latency-critical path where a cudaMalloc,
  * which may synchronise the device, is not allowed.  The pages have no
  * counterpart: this is a packaging of moe_permute, not a step of the method.
- * Arguments, outputs and errors are those of moe_permute, without the
- * workspace.  Its scratch (the per-block expert counts) is a 1 MiB array in
- * the library's static device memory, which every GPU that loads the library
- * holds until the process exits; shapes needing more than that,
- * ceil(T*k / 2048) * E > 262144, return MOE_ERR_UNSUPPORTED.  The first call
- * on a device looks up that array's device address (cudaGetSymbolAddress) and
- * caches it; make that first call before any stream capture.  All calls share
- * the one array, so calls that can overlap on the GPU (unordered streams)
- * race on it.  Nothing in it needs clearing between calls. */
+ * Arguments, outputs and errors are those of moe_permute (the same shape
+ * validation), without the workspace.  Its scratch (the per-block expert
+ * counts) is a 1 MiB array in the library's static device memory, which every
+ * GPU that loads the library holds until the process exits; shapes needing
+ * more than that, ceil(T*k / 2048) * E > 262144, return MOE_ERR_UNSUPPORTED.
+ * The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress) and caches it with the id of the current CUDA
+ * context; a later call that finds another context current (after a device
+ * reset) looks it up again.  Make the first call on a device before any
+ * stream capture.  All calls share the one array, so calls that can overlap
+ * on the GPU (unordered streams) race on it.  Nothing in it needs clearing
+ * between calls: every entry a call reads, that call has written first.  The
+ * call allocates and frees nothing. */
 MOE_API moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_idx,
                                        int32_t* counts, int32_t* offsets, int32_t* perm,
                                        int32_t* inv, int32_t* err_flag, void* stream);
@@ -245,6 +276,110 @@ MOE_API moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x,
  *   y_slots [T*k + S*T, H] dtype, inv [T*k] int32, y [T, H] dtype output. */
 MOE_API moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* inv,
                        void* y, void* stream);
+
+/* Expert parallelism ("Mixture of Experts in Transformers", section "expert
+ * parallelism"): GroupedGemmParallel keeps E/N experts on each of N ranks, a
+ * slice of dim 0 of the packed gate_up_proj and down_proj; RouterParallel maps
+ * the global expert indices to the rank's local ones and masks the other
+ * ranks' experts; the ranks' partial outputs are then summed by an
+ * all-reduce.  Every rank routes and plans the same tokens (moe_route and
+ * moe_permute over all E experts give identical results on every rank), runs
+ * the FFNs of its own experts, combines the slots of its own experts into a
+ * float32 partial, and the partials are summed across ranks (an all-reduce,
+ * for example NCCL's, on the caller's side) before one rounding to dtype.
+ *
+ * moe_forward_experts: moe_forward for routed experts [e_begin, e_end) only.
+ *   gate_up_local [e_end - e_begin, 2I, H], down_local [e_end - e_begin, H, I]:
+ *   the weights of those experts (expert e at index e - e_begin), NULL
+ *   allowed when the range is empty.  sh_gate_up / sh_down: all n_shared
+ *   shared experts, or both NULL on the ranks that do not compute them.
+ *   Writes the y_slots rows of the range, [offsets[e_begin], offsets[e_end]),
+ *   and, with the shared experts, rows T*k ... T*k + S*T - 1; other rows are
+ *   left untouched.  Other arguments, workspace and errors as moe_forward;
+ *   MOE_ERR_INVALID_ARG for a range outside [0, E] or only one shared
+ *   pointer.
+ * moe_combine_experts: the rank's float32 partial
+ *   y_partial[t] = sum over j with e_begin <= topk_idx[t*k+j] < e_end of
+ *                  y_slots[inv[t*k+j]]  (j ascending)
+ *                + (with_shared ? sum_s y_slots[T*k + s*T + t] : 0).
+ *   y_slots [T*k + S*T, H] dtype, inv [T*k], topk_idx [T, k] int32,
+ *   y_partial [T, H] float32 output (16-byte aligned for bf16).
+ * moe_cast_f32: y = y32 rounded once to dtype (round to nearest even); y32
+ *   [T, H] float32 (16-byte aligned), y [T, H] dtype (8-byte aligned). */
+MOE_API moe_status moe_forward_experts(const moe_shape* shape, int32_t e_begin, int32_t e_end,
+                                       const void* x, const int32_t* offsets,
+                                       const int32_t* perm, const float* topk_w,
+                                       const void* gate_up_local, const void* down_local,
+                                       const void* sh_gate_up, const void* sh_down,
+                                       void* y_slots, int32_t* err_flag, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+MOE_API moe_status moe_combine_experts(const moe_shape* shape, int32_t e_begin, int32_t e_end,
+                                       int32_t with_shared, const void* y_slots,
+                                       const int32_t* inv, const int32_t* topk_idx,
+                                       float* y_partial, void* stream);
+MOE_API moe_status moe_cast_f32(const moe_shape* shape, const float* y32, void* y, void* stream);
+
+/* Training: the backward pass of the block.
+ *
+ * The pages name the training side of the block without detailing it: the
+ * PhiMoE page attaches a load-balancing auxiliary loss to the router
+ * ("PhiMoE in Transformers", section 6: load_balancing_loss_func after Switch
+ * Transformer eqs. (4)-(6), times router_aux_loss_coef) and "Mixture of
+ * Experts in Transformers" mentions fast grouped-GEMM training kernels.  The
+ * gradients here are the chain rule through the forward above, for top-k
+ * routing with the softmax over the selected k (the selection itself carries
+ * no gradient):
+ *   slot (t, j), expert e, weight w:  dO = s w dy_t
+ *     dh = Wd_e^T dO,  dg = dh * u * SiLU'(g),  du = dh * SiLU(g)
+ *     dWd_e += dO h^T,  dWgu_e += [dg; du] x_t^T,  dx_t += Wgu_e^T [dg; du]
+ *     dw = s <dy_t, FFN_e(x_t)>
+ *   router: dl_tj = w_tj (dw_tj - sum_i w_ti dw_ti) on the selected experts,
+ *     plus, when aux_coef != 0, the auxiliary loss
+ *     coef * E * sum_e f_e P_e (f_e = tokens dispatched to e / T, P_e = mean
+ *     softmax probability of e over all E logits):
+ *     dl_te += coef E / T * p_te (f_e - sum_c p_tc f_c);
+ *     dWr = dl^T x, d_bias = sum_t dl_t, dx_t += dl_t Wr
+ *   shared experts: as a routed expert with weight 1 on every token.
+ * Supported: bf16, T > 8 (the tensor-core path), H a multiple of 64, I and
+ * I_shared multiples of 32; otherwise MOE_ERR_UNSUPPORTED.
+ *
+ * moe_train_state_size: bytes of the state moe_forward_train keeps for the
+ *   backward pass (gate/up pre-activations, SwiGLU outputs and the gathered x
+ *   rows, bf16).
+ * moe_forward_train: moe_forward that also fills `state` (>= that size,
+ *   16-byte aligned); y_slots as moe_forward.
+ * moe_backward_workspace_size / moe_backward: with the forward's routing
+ *   (topk_idx, topk_w, counts, offsets, perm, inv), weights, `state` and the
+ *   upstream gradient dy [T, H] bf16, writes
+ *     dx [T, H] bf16,
+ *     d_gate_up [E, 2I, H], d_down [E, H, I], d_sh_gate_up [S, 2Is, H],
+ *     d_sh_down [S, H, Is], d_w_router [E, H] float32 (overwritten, not
+ *     accumulated), d_router_bias [E] float32 or NULL,
+ *     d_topk_w [T, k] float32 or NULL (the routing weights' gradient),
+ *     aux_loss [1] float32 or NULL (the auxiliary loss value; accumulated
+ *     with atomics, so its last bits may vary run to run).
+ *   logits [T, E] float32 (the router's, from moe_route) is needed only when
+ *   aux_coef != 0.  Every other output is deterministic.  Workspace: at least
+ *   moe_backward_workspace_size() bytes, 16-byte aligned. */
+MOE_API moe_status moe_train_state_size(const moe_shape* shape, size_t* bytes);
+MOE_API moe_status moe_forward_train(const moe_shape* shape, const void* x,
+                                     const int32_t* offsets, const int32_t* perm,
+                                     const float* topk_w, const void* gate_up, const void* down,
+                                     const void* sh_gate_up, const void* sh_down, void* y_slots,
+                                     void* state, size_t state_bytes, int32_t* err_flag,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+MOE_API moe_status moe_backward_workspace_size(const moe_shape* shape, size_t* bytes);
+MOE_API moe_status moe_backward(const moe_shape* shape, const void* x, const float* w_router,
+                                const int32_t* topk_idx, const float* topk_w,
+                                const int32_t* counts, const int32_t* offsets,
+                                const int32_t* perm, const int32_t* inv, const void* gate_up,
+                                const void* down, const void* sh_gate_up, const void* sh_down,
+                                const void* state, const float* logits, float aux_coef,
+                                const void* dy, void* dx, float* d_gate_up, float* d_down,
+                                float* d_sh_gate_up, float* d_sh_down, float* d_w_router,
+                                float* d_router_bias, float* d_topk_w, float* aux_loss,
+                                int32_t* err_flag, void* workspace, size_t workspace_bytes,
+                                void* stream);
 
 /* Diagnostic with no counterpart in the pages: runs the bounded pipeline wait
  * that every kernel here uses on an mbarrier nothing ever arrives on, so that

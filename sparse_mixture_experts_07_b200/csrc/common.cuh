@@ -17,6 +17,25 @@ constexpr int kMaxShared = 8;
 constexpr int kMaxK = 16;
 constexpr int kMaxGroups = kMaxExperts + kMaxShared;
 
+// Host-side validation of a moe_shape, common to every entry point of the C
+// ABI (defined in moe_api.cu): MOE_ERR_INVALID_ARG for inconsistent sizes,
+// MOE_ERR_UNSUPPORTED for sizes outside what the kernels implement.
+moe_status check_shape(const moe_shape* s);
+
+// Workspace buffers of the backward pass (backward.cu); rows of the padded
+// sorted order (P rows: each expert's rows padded to a multiple of 128).
+struct BackwardBuffers {
+    int32_t* poffsets;   // [E+1] padded expert offsets
+    void* dO;            // [P, H] routed output gradients; later dX of the slots
+    void* dgu;           // [P, 2I] gradients of the gate and up pre-activations
+    void* dgu_sh;        // [S*T, 2Is] the same for the shared experts
+    void* dX_sh;         // [S*T, H] the shared experts' input gradients
+    float* dw_raw;       // [T*k, n-tiles] parts of the routing-weight gradients x weight
+    float* dl;           // [T, E] logit gradients
+    float* part;         // [chunks, E, H] router weight gradient partials
+    float* partb;        // [chunks, E] router bias gradient partials
+};
+
 // Device-detected faults are OR-ed into the caller's err_flag as 1 << status.
 __device__ __forceinline__ void raise_error(int32_t* err_flag, int status) {
     if (err_flag) atomicOr(err_flag, 1 << status);

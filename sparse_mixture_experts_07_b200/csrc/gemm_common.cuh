@@ -27,7 +27,29 @@ struct GemmParams {
     int group_m;
     int32_t* err_flag;
     uint64_t timeout_ns;
+    // kSwiGLU, training forward: also store the pre-activations [g | u] of
+    // every row (bf16, row stride 2N) for the backward pass; NULL: do not
+    void* gu_routed;
+    void* gu_shared;
 };
+
+// Stores 32 gate and 32 up values of one row as bf16 into gu (row stride 2N,
+// gate at column n, up at N + n), 16-byte vectors, columns < N only.
+__device__ __forceinline__ void store_gu32(__nv_bfloat16* gu_row, int n, int N,
+                                           const float (&gv)[32], const float (&uv)[32]) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        if (n + 8 * v >= N) break;
+        uint32_t g4[4], u4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            g4[j] = pack_bf16x2(gv[8 * v + 2 * j], gv[8 * v + 2 * j + 1]);
+            u4[j] = pack_bf16x2(uv[8 * v + 2 * j], uv[8 * v + 2 * j + 1]);
+        }
+        *reinterpret_cast<uint4*>(gu_row + n + 8 * v) = make_uint4(g4[0], g4[1], g4[2], g4[3]);
+        *reinterpret_cast<uint4*>(gu_row + N + n + 8 * v) = make_uint4(u4[0], u4[1], u4[2], u4[3]);
+    }
+}
 
 struct TileCoord {
     int g;          // group

@@ -234,6 +234,9 @@ __global__ void __launch_bounds__(sm100::THREADS, 1) grouped_gemm_sm100(
                             if (n + 8 * v < N)
                                 dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1],
                                                     packed[4 * v + 2], packed[4 * v + 3]);
+                        __nv_bfloat16* gu = static_cast<__nv_bfloat16*>(c.routed ? p.gu_routed
+                                                                                  : p.gu_shared);
+                        if (gu) store_gu32(gu + orow * 2 * N, n, N, gv, uv);
                     }
                 }
             } else {
@@ -285,7 +288,8 @@ cudaError_t launch_ffn_sm100(const moe_shape& s, const void* x, const void* x_pe
                              const int32_t* offsets, const int32_t* perm, const float* topk_w,
                              const void* gate_up, const void* down, const void* sh_gate_up,
                              const void* sh_down, void* h_routed, void* h_shared, void* y_slots,
-                             int32_t* err_flag, int num_sms, int group_m, cudaStream_t st) {
+                             int32_t* err_flag, int num_sms, int group_m, cudaStream_t st,
+                             void* gu_routed, void* gu_shared) {
     using namespace sm100;
     const int64_t Tk = s.T * s.k;
     const int S = s.n_shared;
@@ -319,6 +323,8 @@ cudaError_t launch_ffn_sm100(const moe_shape& s, const void* x, const void* x_pe
     p.group_m = group_m;
     p.err_flag = err_flag;
     p.timeout_ns = 4000000000ull;
+    p.gu_routed = gu_routed;
+    p.gu_shared = gu_shared;
 
     const int64_t mt_bound = ceil_div(Tk, BM) + s.E;
     const int64_t mt_shared = S > 0 ? S * ceil_div(s.T, BM) : 0;
@@ -349,6 +355,8 @@ cudaError_t launch_ffn_sm100(const moe_shape& s, const void* x, const void* x_pe
     if (e != cudaSuccess) return e;
 
     // GEMM 2
+    p.gu_routed = nullptr;
+    p.gu_shared = nullptr;
     p.n_tiles_routed = static_cast<int>(ceil_div(s.H, BN));
     p.n_tiles_shared = p.n_tiles_routed;
     p.K_routed = s.I;

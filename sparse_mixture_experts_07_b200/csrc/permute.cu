@@ -341,12 +341,14 @@ cudaError_t launch_permute(const moe_shape& s, const int32_t* idx, int32_t* coun
 //
 // Host code must not pass `g_permute_scratch` itself to a kernel: on the host
 // that name is only a stand-in, not a device address.  The device address is
-// looked up once per device with cudaGetSymbolAddress, on the first call made
-// while that device is current, and cached; make that first call before any
-// stream capture.  The array keeps the last call's contents; the histogram
-// kernel overwrites every entry it later reads, so nothing needs clearing.
-// All calls share the one array: calls whose kernels may overlap on the GPU
-// (different streams without ordering between them) race on it.
+// looked up with cudaGetSymbolAddress on the first call made while a device is
+// current, and cached together with the id of the CUDA context it belongs to;
+// a call that finds a different context current (the device was reset since)
+// looks it up again.  Make the first call on a device before any stream
+// capture.  The array keeps the last call's contents; the histogram kernel
+// overwrites every entry it later reads, so nothing needs clearing.  All calls
+// share the one array: calls whose kernels may overlap on the GPU (different
+// streams without ordering between them) race on it.
 #include <mutex>
 
 namespace moe {
@@ -358,23 +360,61 @@ static __device__ __align__(256) int32_t g_permute_scratch[moe::kNoallocScratchI
 
 namespace {
 
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[moe::kNoallocMaxDevices] = {nullptr};
+struct ScratchEntry {
+    void* ptr;
+    unsigned long long ctx_id;
+};
 
-// Device address of g_permute_scratch on the current device (looked up once).
+std::mutex g_scratch_mu;
+ScratchEntry g_scratch[moe::kNoallocMaxDevices] = {};
+
+// Id of the current CUDA context (driver entry points cuCtxGetCurrent and
+// cuCtxGetId); 0 when it cannot be determined, which disables the cache.
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrentFn)(CUcontext*);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        void* a = nullptr;
+        void* b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) ==
+                cudaSuccess && qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<GetCurrentFn>(a);
+            get_id = reinterpret_cast<GetIdFn>(b);
+        }
+        looked_up = true;
+    }
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_permute_scratch in the current device's context.
 cudaError_t noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= moe::kNoallocMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    // 0 before the runtime has made a context current: then look the address
+    // up, which initialises the context, and read the id afterwards
+    const unsigned long long ctx = current_context_id();
+    ScratchEntry& entry = g_scratch[dev];
+    if (!entry.ptr || ctx == 0 || entry.ctx_id != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_permute_scratch);
         if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
+        entry.ptr = p;
+        entry.ctx_id = current_context_id();
     }
-    *out = g_scratch_ptr[dev];
+    *out = entry.ptr;
     return cudaSuccess;
 }
 
@@ -383,14 +423,10 @@ cudaError_t noalloc_scratch(void** out) {
 extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_idx,
                                           int32_t* counts, int32_t* offsets, int32_t* perm,
                                           int32_t* inv, int32_t* err_flag, void* stream) {
-    if (!shape) return MOE_ERR_INVALID_ARG;
+    // the same validation as moe_permute, then the scratch limit
+    const moe_status st = moe::check_shape(shape);
+    if (st != MOE_OK) return st;
     const moe_shape& s = *shape;
-    if (s.T < 0 || s.H <= 0 || s.I <= 0 || s.E <= 0 || s.k <= 0 || s.k > s.E ||
-        s.n_shared < 0 || (s.n_shared > 0 && s.I_shared <= 0) ||
-        (s.dtype != MOE_F32 && s.dtype != MOE_BF16))
-        return MOE_ERR_INVALID_ARG;
-    if (s.E > moe::kMaxExperts || s.k > moe::kMaxK || s.T * s.k >= (int64_t(1) << 31))
-        return MOE_ERR_UNSUPPORTED;
     if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
     if (s.T > 0 && (!topk_idx || !perm || !inv)) return MOE_ERR_INVALID_ARG;
     // the plan needs ceil(T*k / 2048) * E ints of scratch

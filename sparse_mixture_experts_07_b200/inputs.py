@@ -8,7 +8,9 @@ router's affine map in float64, only to choose inputs:
 * near-tie rejection: a token row is redrawn until, on the exact stored values,
   its (k)-th and (k+1)-th largest router scores differ by more than 1e-3 and the
   k largest are pairwise more than 1e-3 apart, so that the expert selection and
-  its order cannot depend on the rounding of either implementation;
+  its order cannot depend on the rounding of either implementation (for
+  DeepSeek-V3 routing the scores are sigmoid(logit) + bias, and the kept and
+  first dropped group scores must be 1e-3 apart as well);
 * Zipf load calibration: a per-expert router bias is fitted so that the share
   of tokens routed to expert e follows a Zipf law (the gpt-oss- and
   DeepSeek-V3-shaped workloads).
@@ -52,6 +54,12 @@ class MoEConfig:
     routed_scale: float = 1.0
     dtype: str = "bf16"    # activations and expert weights: "bf16" or "f32"
     zipf_s: Optional[float] = None   # None: unbiased router
+    # "softmax": top-k of the (biased) logits, softmax over the k; "noaux_tc":
+    # DeepSeek-V3 routing (sigmoid scores, bias in the selection only, the k
+    # experts drawn from the topk_group best of n_group expert groups)
+    routing: str = "softmax"
+    n_group: int = 1
+    topk_group: int = 1
 
     @property
     def slots(self) -> int:
@@ -76,6 +84,11 @@ CONFIGS = {
     "gptoss": MoEConfig("gptoss", T=16384, H=2880, I=2880, E=32, k=4, zipf_s=1.0),
     "dsv3": MoEConfig("dsv3", T=32768, H=2048, I=1024, E=64, k=6, n_shared=2,
                       I_shared=1024, routed_scale=2.5, zipf_s=1.2),
+    # the same layer with the DeepSeek-V3 routing the Instella page names
+    # (noaux_tc); 8 groups with 4 kept, DeepSeek-V3's published values
+    "dsv3_noaux": MoEConfig("dsv3_noaux", T=32768, H=2048, I=1024, E=64, k=6, n_shared=2,
+                            I_shared=1024, routed_scale=2.5, zipf_s=1.2, routing="noaux_tc",
+                            n_group=8, topk_group=4),
 }
 
 
@@ -117,6 +130,35 @@ def _bad_rows(scores: np.ndarray, k: int) -> np.ndarray:
     if gaps.shape[1] == 0:
         return np.zeros(scores.shape[0], dtype=bool)
     return (gaps <= GAP).any(axis=1)
+
+
+def _sigmoid64(v: np.ndarray) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-v))
+
+
+def _noaux_bad_rows(logits: np.ndarray, bias: Optional[np.ndarray], k: int, n_group: int,
+                    topk_group: int) -> np.ndarray:
+    """Rows whose noaux_tc decisions have a near tie (gap <= GAP): between the
+    kept and the first dropped group score, or among the k + 1 largest
+    selection scores of the kept groups."""
+    T, E = logits.shape
+    c = _sigmoid64(logits) + (0.0 if bias is None else bias.astype(np.float64)[None, :])
+    gsize = E // n_group
+    gs = np.sort(c.reshape(T, n_group, gsize), axis=2)[:, :, -min(2, gsize):].sum(axis=2)
+    order = np.argsort(-gs, axis=1)
+    gsorted = np.take_along_axis(gs, order, axis=1)
+    bad = np.zeros(T, dtype=bool)
+    if topk_group < n_group:
+        bad |= gsorted[:, topk_group - 1] - gsorted[:, topk_group] <= GAP
+    keep = np.zeros((T, n_group), dtype=bool)
+    np.put_along_axis(keep, order[:, :topk_group], True, axis=1)
+    allowed = np.repeat(keep, gsize, axis=1)
+    cm = np.where(allowed, c, -np.inf)
+    m = min(k + 1, topk_group * gsize)
+    top = -np.sort(-cm, axis=1)[:, :m]
+    if m > 1:
+        bad |= (top[:, :-1] - top[:, 1:] <= GAP).any(axis=1)
+    return bad
 
 
 def _loads(scores: np.ndarray, k: int) -> np.ndarray:
@@ -179,16 +221,23 @@ def make_inputs(cfg: MoEConfig, seed: int = 0, weights_device: str = "cpu",
     wr = torch.randn(E, H, generator=g) * INIT_STD
     wr_np = wr.numpy()
 
+    noaux = cfg.routing == "noaux_tc"
     bias_np = None
     target = None
     if cfg.zipf_s is not None:
         target = zipf_targets(E, k, cfg.zipf_s)
-        bias_np = calibrate_bias(_scores64(x.float().numpy(), wr_np, None), k, target)
+        base = _scores64(x.float().numpy(), wr_np, None)
+        # noaux_tc selects on sigmoid(logit) + bias (the fit ignores the groups)
+        bias_np = calibrate_bias(_sigmoid64(base) if noaux else base, k, target)
         bias_np = bias_np.astype(np.float32)
 
     redrawn = 0
     for _ in range(max_redraw_rounds):
-        bad = _bad_rows(_scores64(x.float().numpy(), wr_np, bias_np), k)
+        if noaux:
+            bad = _noaux_bad_rows(_scores64(x.float().numpy(), wr_np, None), bias_np, k,
+                                  cfg.n_group, cfg.topk_group)
+        else:
+            bad = _bad_rows(_scores64(x.float().numpy(), wr_np, bias_np), k)
         nbad = int(bad.sum())
         if nbad == 0:
             break

@@ -21,7 +21,9 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_INDEX", 6: "MOE_ERR_TIMEOUT"}
 EXPORTS = ("moe_status_str", "moe_workspace_size", "moe_route", "moe_permute", "moe_forward",
            "moe_combine", "moe_router_split_size", "moe_router_split", "moe_route_split",
-           "moe_forward_mxfp4")
+           "moe_forward_mxfp4", "moe_forward_experts", "moe_combine_experts", "moe_cast_f32",
+           "moe_route_noaux_tc", "moe_train_state_size", "moe_forward_train",
+           "moe_backward_workspace_size", "moe_backward")
 
 
 class MoEShape(ctypes.Structure):
@@ -62,6 +64,19 @@ def load_library(path: str = LIB_PATH):
     lib.moe_router_split.argtypes = [S, P, P, ctypes.c_size_t, P]
     lib.moe_route_split.argtypes = [S, P, P, P, P, P, P, P, P, P]
     lib.moe_forward_mxfp4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    i32 = ctypes.c_int32
+    lib.moe_forward_experts.argtypes = [S, i32, i32, P, P, P, P, P, P, P, P, P, P, P,
+                                        ctypes.c_size_t, P]
+    lib.moe_combine_experts.argtypes = [S, i32, i32, i32, P, P, P, P, P]
+    lib.moe_cast_f32.argtypes = [S, P, P, P]
+    lib.moe_route_noaux_tc.argtypes = [S, i32, i32, P, P, P, P, P, P, P, P, P]
+    sz = ctypes.POINTER(ctypes.c_size_t)
+    lib.moe_train_state_size.argtypes = [S, sz]
+    lib.moe_forward_train.argtypes = [S, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P,
+                                      ctypes.c_size_t, P]
+    lib.moe_backward_workspace_size.argtypes = [S, sz]
+    lib.moe_backward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_float, P,
+                                 P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     for f in EXPORTS[1:]:
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -160,6 +175,24 @@ def route(shape: Shape, x, w_router, router_bias=None, logits=False, out=None, s
     return idx, w, lg
 
 
+def route_noaux_tc(shape: Shape, x, w_router, score_bias, n_group: int, topk_group: int,
+                   out=None, logits=None, stream=None, err_flag=None, w_split=None):
+    """DeepSeek-V3 ("noaux_tc") routing: (topk_idx [T,k] int32, topk_w [T,k]
+    f32, logits [T,E] f32).  `score_bias` steers the selection only."""
+    lib = load_library()
+    dev = x.device
+    idx = out["topk_idx"] if out else torch.empty(shape.T, shape.k, dtype=torch.int32, device=dev)
+    w = out["topk_w"] if out else torch.empty(shape.T, shape.k, dtype=torch.float32, device=dev)
+    if logits is None:
+        logits = torch.empty(shape.T, shape.E, dtype=torch.float32, device=dev)
+    _check(lib.moe_route_noaux_tc(ctypes.byref(shape.c()), n_group, topk_group, _ptr(x),
+                                  _ptr(w_router), _ptr(w_split), _ptr(score_bias), _ptr(logits),
+                                  _ptr(idx), _ptr(w), _ptr(err_flag), _stream(stream)),
+           "moe_route_noaux_tc", "moe_train_state_size", "moe_forward_train",
+           "moe_backward_workspace_size", "moe_backward")
+    return idx, w, logits
+
+
 def permute(shape: Shape, topk_idx, workspace, err_flag, out=None, stream=None):
     """(counts [E], offsets [E+1], perm [T*k], inv [T*k]) int32."""
     lib = load_library()
@@ -207,6 +240,44 @@ def forward_mxfp4(shape: Shape, x, offsets, perm, topk_w, mxfp4: dict, workspace
     return y_slots
 
 
+def forward_experts(shape: Shape, e_begin: int, e_end: int, x, offsets, perm, topk_w,
+                    gate_up_local, down_local, sh_gate_up, sh_down, workspace, err_flag,
+                    y_slots, stream=None):
+    """The expert FFNs of routed experts [e_begin, e_end) (their weights only),
+    plus the shared experts when sh_gate_up / sh_down are given; writes those
+    experts' rows of y_slots."""
+    lib = load_library()
+    _check(lib.moe_forward_experts(ctypes.byref(shape.c()), e_begin, e_end, _ptr(x),
+                                   _ptr(offsets), _ptr(perm), _ptr(topk_w), _ptr(gate_up_local),
+                                   _ptr(down_local), _ptr(sh_gate_up), _ptr(sh_down),
+                                   _ptr(y_slots), _ptr(err_flag), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "moe_forward_experts")
+    return y_slots
+
+
+def combine_experts(shape: Shape, e_begin: int, e_end: int, with_shared: bool, y_slots, inv,
+                    topk_idx, y_partial=None, stream=None):
+    """float32 partial [T, H]: the slots of experts [e_begin, e_end) in token
+    order (plus the shared experts' rows when with_shared)."""
+    lib = load_library()
+    if y_partial is None:
+        y_partial = torch.empty(shape.T, shape.H, dtype=torch.float32, device=y_slots.device)
+    _check(lib.moe_combine_experts(ctypes.byref(shape.c()), e_begin, e_end, int(with_shared),
+                                   _ptr(y_slots), _ptr(inv), _ptr(topk_idx), _ptr(y_partial),
+                                   _stream(stream)), "moe_combine_experts")
+    return y_partial
+
+
+def cast_f32(shape: Shape, y32, y=None, stream=None):
+    """y [T, H] (dtype) = y32 rounded once."""
+    lib = load_library()
+    if y is None:
+        y = torch.empty(shape.T, shape.H, dtype=shape.torch_dtype, device=y32.device)
+    _check(lib.moe_cast_f32(ctypes.byref(shape.c()), _ptr(y32), _ptr(y), _stream(stream)),
+           "moe_cast_f32")
+    return y
+
+
 def combine(shape: Shape, y_slots, inv, y=None, stream=None):
     """y [T, H] (dtype)."""
     lib = load_library()
@@ -215,6 +286,70 @@ def combine(shape: Shape, y_slots, inv, y=None, stream=None):
     _check(lib.moe_combine(ctypes.byref(shape.c()), _ptr(y_slots), _ptr(inv), _ptr(y),
                            _stream(stream)), "moe_combine")
     return y
+
+
+def train_state_size(shape: Shape) -> int:
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    _check(lib.moe_train_state_size(ctypes.byref(shape.c()), ctypes.byref(n)),
+           "moe_train_state_size")
+    return n.value
+
+
+def backward_workspace_size(shape: Shape) -> int:
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    _check(lib.moe_backward_workspace_size(ctypes.byref(shape.c()), ctypes.byref(n)),
+           "moe_backward_workspace_size")
+    return n.value
+
+
+def forward_train(shape: Shape, x, offsets, perm, topk_w, gate_up, down, sh_gate_up, sh_down,
+                  workspace, state, err_flag, y_slots=None, stream=None):
+    """moe_forward that also keeps, in `state`, what moe_backward reads."""
+    lib = load_library()
+    if y_slots is None:
+        y_slots = torch.empty(shape.slot_rows, shape.H, dtype=shape.torch_dtype, device=x.device)
+    _check(lib.moe_forward_train(ctypes.byref(shape.c()), _ptr(x), _ptr(offsets), _ptr(perm),
+                                 _ptr(topk_w), _ptr(gate_up), _ptr(down), _ptr(sh_gate_up),
+                                 _ptr(sh_down), _ptr(y_slots), _ptr(state), state.numel(),
+                                 _ptr(err_flag), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "moe_forward_train")
+    return y_slots
+
+
+def backward(shape: Shape, x, w_router, topk_idx, topk_w, counts, offsets, perm, inv, gate_up,
+             down, sh_gate_up, sh_down, state, dy, workspace, err_flag, logits=None,
+             aux_coef: float = 0.0, want_topk_w_grad=False, want_aux_loss=False, stream=None):
+    """The block's gradients: dict of dx (dtype), gate_up, down, sh_gate_up,
+    sh_down, w_router, router_bias (float32), and topk_w / aux_loss if asked."""
+    lib = load_library()
+    dev = x.device
+    f32 = torch.float32
+    E, H, I, S = shape.E, shape.H, shape.I, shape.n_shared
+    Is = shape.I_shared if S else 0
+    g = {
+        "x": torch.empty(shape.T, H, dtype=shape.torch_dtype, device=dev),
+        "gate_up": torch.empty(E, 2 * I, H, dtype=f32, device=dev),
+        "down": torch.empty(E, H, I, dtype=f32, device=dev),
+        "sh_gate_up": torch.empty(S, 2 * Is, H, dtype=f32, device=dev) if S else None,
+        "sh_down": torch.empty(S, H, Is, dtype=f32, device=dev) if S else None,
+        "w_router": torch.empty(E, H, dtype=f32, device=dev),
+        "router_bias": torch.empty(E, dtype=f32, device=dev),
+        "topk_w": torch.empty(shape.T, shape.k, dtype=f32, device=dev) if want_topk_w_grad
+        else None,
+        "aux_loss": torch.zeros(1, dtype=f32, device=dev) if want_aux_loss else None,
+    }
+    _check(lib.moe_backward(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(topk_idx),
+                            _ptr(topk_w), _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
+                            _ptr(gate_up), _ptr(down), _ptr(sh_gate_up), _ptr(sh_down),
+                            _ptr(state), _ptr(logits), float(aux_coef), _ptr(dy), _ptr(g["x"]),
+                            _ptr(g["gate_up"]), _ptr(g["down"]), _ptr(g["sh_gate_up"]),
+                            _ptr(g["sh_down"]), _ptr(g["w_router"]), _ptr(g["router_bias"]),
+                            _ptr(g["topk_w"]), _ptr(g["aux_loss"]), _ptr(err_flag),
+                            _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_backward")
+    return g
 
 
 class MoELayer:
@@ -226,11 +361,17 @@ class MoELayer:
     """
 
     def __init__(self, shape: Shape, w_router, router_bias, gate_up=None, down=None,
-                 sh_gate_up=None, sh_down=None, mxfp4=None):
+                 sh_gate_up=None, sh_down=None, mxfp4=None, routing=None):
         """Expert weights either as gate_up / down (dtype of `shape`), or as
-        `mxfp4` = {gate_up_q, gate_up_s, down_q, down_s} (decode batches)."""
+        `mxfp4` = {gate_up_q, gate_up_s, down_q, down_s} (decode batches).
+        `routing`: None for top-k with a softmax over the selected k (the bias
+        added to the logits), or ("noaux_tc", n_group, topk_group) for
+        DeepSeek-V3 routing (the bias steers the selection only)."""
         self.shape = shape
         self.mxfp4 = mxfp4
+        self.routing = routing
+        if routing is not None and routing[0] != "noaux_tc":
+            raise ValueError(f"unknown routing {routing!r}")
         self.w_router, self.router_bias = w_router, router_bias
         # split once here, at load time; refresh it if w_router changes
         self.w_split = router_split(shape, w_router)
@@ -250,12 +391,20 @@ class MoELayer:
             "y_slots": torch.empty(shape.slot_rows, H, dtype=shape.torch_dtype, device=dev),
             "y": torch.empty(T, H, dtype=shape.torch_dtype, device=dev),
         }
+        if routing is not None:
+            self.buf["logits"] = torch.empty(T, E, dtype=torch.float32, device=dev)
         self.last = None
 
     def __call__(self, x, stream=None, y=None):
         s, b = self.shape, self.buf
-        idx, w, _ = route(s, x, self.w_router, self.router_bias, out=b, stream=stream,
-                          err_flag=self.err_flag, w_split=self.w_split)
+        if self.routing is not None:
+            idx, w, _ = route_noaux_tc(s, x, self.w_router, self.router_bias, self.routing[1],
+                                       self.routing[2], out=b, logits=b["logits"],
+                                       stream=stream, err_flag=self.err_flag,
+                                       w_split=self.w_split)
+        else:
+            idx, w, _ = route(s, x, self.w_router, self.router_bias, out=b, stream=stream,
+                              err_flag=self.err_flag, w_split=self.w_split)
         counts, offsets, perm, inv = permute(s, idx, self.workspace, self.err_flag, out=b,
                                              stream=stream)
         if self.mxfp4 is not None:

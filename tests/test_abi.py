@@ -160,7 +160,7 @@ def test_forward_mxfp4_argument_checks(lib):
     def call(shape, ws_bytes=need, x=ok, q=ok, ws=ok):
         return lib.moe_forward_mxfp4(ctypes.byref(shape), x, ok, ok, ok, q, ok, ok, ok, ok,
                                      None, ws, ws_bytes, None)
-    assert call(_shape(T=9, H=256, I=128)) == 2              # decode batches only
+    assert call(_shape(T=65, H=256, I=128)) == 2             # decode batches only (T <= 64)
     assert call(_shape(T=4, H=256, I=128, n_shared=1, I_shared=64)) == 2
     assert call(_shape(T=4, H=136, I=128)) == 2              # H not a multiple of 32
     assert call(_shape(T=4, H=256, I=136)) == 2
@@ -170,6 +170,9 @@ def test_forward_mxfp4_argument_checks(lib):
     assert call(s, ws_bytes=need - 1) == 3
     assert call(s, ws=None) == 3
     assert call(s, x=ctypes.c_void_p(4096 + 8)) == 2
+    # scale arrays are read in aligned 4-byte words
+    assert lib.moe_forward_mxfp4(ctypes.byref(s), ok, ok, ok, ok, ok, ctypes.c_void_p(4096 + 2),
+                                 ok, ok, ok, None, ok, need, None) == 2
     assert call(_shape(T=0, H=256, I=128), x=None, q=None, ws=None, ws_bytes=0) == 0
 
 
@@ -191,3 +194,35 @@ def test_missing_library_fails_loudly(tmp_path):
             m.load_library(str(tmp_path / "libmoe.so"))
     finally:
         m._lib = saved
+
+
+@pytest.mark.parametrize("kw", [
+    dict(k=9), dict(E=0), dict(T=-1), dict(dtype=7), dict(n_shared=1, I_shared=0),
+    dict(E=300, k=2), dict(n_shared=9, I_shared=64), dict(H=100), dict(I=100),
+    dict(n_shared=1, I_shared=36), dict(T=1 << 30, k=2, n_shared=2, I_shared=64),
+])
+def test_noalloc_permute_validates_shapes_like_permute(lib, kw):
+    """moe_permute_noalloc applies moe_permute's shape checks (before its own
+    scratch limit), so both return the same status on an invalid shape."""
+    s = _shape(**kw)
+    p = ctypes.c_void_p(256)     # never dereferenced: validation fails first
+    lib.moe_permute_noalloc.argtypes = [ctypes.POINTER(MoEShape)] + [ctypes.c_void_p] * 7
+    lib.moe_permute_noalloc.restype = ctypes.c_int
+    want = lib.moe_permute(ctypes.byref(s), p, p, p, p, p, None, p, 1 << 40, None)
+    got = lib.moe_permute_noalloc(ctypes.byref(s), p, p, p, p, p, None, None)
+    assert want != 0 and got == want
+
+
+@pytest.mark.parametrize("n_group,topk_group", [(3, 1), (4, 0), (4, 5), (8, 1), (64, 1), (0, 1)])
+def test_noaux_rejects_bad_group_arguments(lib, n_group, topk_group):
+    """E % n_group != 0, topk_group outside [1, n_group], k above the kept
+    experts, n_group above 32: MOE_ERR_INVALID_ARG before any launch."""
+    s = _shape(T=4, E=16, k=4)
+    p = ctypes.c_void_p(256)
+    f = lib.moe_route_noaux_tc
+    f.argtypes = [ctypes.POINTER(MoEShape), ctypes.c_int32, ctypes.c_int32] + \
+        [ctypes.c_void_p] * 9
+    f.restype = ctypes.c_int
+    assert f(ctypes.byref(s), n_group, topk_group, p, p, None, None, p, p, p, None, None) == 1
+    # valid groups, but the logits buffer the selection reads is required
+    assert f(ctypes.byref(s), 4, 2, p, p, None, None, None, p, p, None, None) == 1
