@@ -188,8 +188,7 @@ def route_noaux_tc(shape: Shape, x, w_router, score_bias, n_group: int, topk_gro
     _check(lib.moe_route_noaux_tc(ctypes.byref(shape.c()), n_group, topk_group, _ptr(x),
                                   _ptr(w_router), _ptr(w_split), _ptr(score_bias), _ptr(logits),
                                   _ptr(idx), _ptr(w), _ptr(err_flag), _stream(stream)),
-           "moe_route_noaux_tc", "moe_train_state_size", "moe_forward_train",
-           "moe_backward_workspace_size", "moe_backward")
+           "moe_route_noaux_tc")
     return idx, w, logits
 
 

@@ -24,17 +24,36 @@ def logit_tol(H: int, logits: np.ndarray) -> float:
     return 2.0 * (H / 16.0) * 2.0 ** -23 * float(np.abs(logits).max()) + 1e-6
 
 
-# Probabilistic per-logit bound: C_LOGIT * sqrt(H/16) * 2^-23 * (sum_h |x_h w_eh| + |b_e|).
-# The H/16 float32 roundings of a 16-product MMA step are independent and of
-# either sign, so their sum grows like the square root of their number; each
-# is at most 2^-23 of the magnitudes summed so far, which sum_h |x_h w_eh|
-# bounds.  C_LOGIT = 1 (the scale alone); see the measured ratios printed by
-# check_routing.
-C_LOGIT = None
+# Probabilistic per-logit bound, checked element by element:
+#   |l_gpu - l| <= C_LOGIT * sqrt(n) * 2^-23 * (sum_h |x_h w_eh| + |b_e|)
+# where n is the number of float32 roundings in the router's accumulation
+# chain.  The products are exact (bf16 x times the bf16 terms of w, or float32
+# FMA); each rounding is at most 2^-23 of the magnitudes summed so far, which
+# sum_h |x_h w_eh| bounds; the roundings are independent and of either sign,
+# so their sum grows like sqrt(n).  n per router path (router_chain_length):
+#   tensor cores (bf16, T > 256, E <= 64): one rounding per 16-product MMA step,
+#     n = H / 16;
+#   one CTA per token (T <= 256): per-lane chains of H / 32, then a 5-level
+#     warp tree, n = H / 32 + 5;
+#   CUDA-core tiled router (float32 x, or E > 64): sequential FMA chains, n = H.
+# C_LOGIT = 1.  Measured on a B200, the largest ratio of the error to this
+# bound over every configuration of the GPU suite is 0.35 (gpt-oss- and
+# DeepSeek-shaped layers, tensor cores; the Mixtral-shaped layer 0.31).
+C_LOGIT = 1.0
 
 
-def logit_scale(x, w_router, bias) -> np.ndarray:
-    """sqrt(H/16) * 2^-23 * (sum_h |x_h w_eh| + |b_e|) for every (token, expert)."""
+def router_chain_length(cfg) -> float:
+    """Float32 roundings in one logit's accumulation on the path moe_route /
+    moe_route_split takes for this configuration."""
+    if cfg.T <= 256:
+        return cfg.H / 32.0 + 5.0
+    if cfg.dtype == "bf16" and cfg.E <= 64:
+        return cfg.H / 16.0
+    return float(cfg.H)
+
+
+def logit_scale(x, w_router, bias, n_chain: float) -> np.ndarray:
+    """sqrt(n_chain) * 2^-23 * (sum_h |x_h w_eh| + |b_e|) for every (token, expert)."""
     xa = np.abs(x.float().numpy().astype(np.float64) if hasattr(x, "float") else np.asarray(x))
     wa = np.abs(w_router.float().numpy().astype(np.float64) if hasattr(w_router, "float")
                 else np.asarray(w_router))
@@ -42,8 +61,7 @@ def logit_scale(x, w_router, bias) -> np.ndarray:
     if bias is not None:
         b = bias.float().numpy() if hasattr(bias, "float") else np.asarray(bias)
         s = s + np.abs(b.astype(np.float64))[None, :]
-    H = wa.shape[1]
-    return np.sqrt(H / 16.0) * 2.0 ** -23 * s
+    return np.sqrt(n_chain) * 2.0 ** -23 * s
 
 
 # Softmax over the selected k: |dw_i| <= w_i (|dl_i| + sum_j w_j |dl_j|) <= 2 max|dl|.
@@ -89,9 +107,9 @@ def tolerance(cfg: MoEConfig) -> float:
 
 
 def check_routing(cfg: MoEConfig, inp: dict, res: dict, tokens=None):
-    """Indices and plan bit-exact; logits within C_LOGIT times the per-logit
-    scale (and the worst-case ceiling); weights within twice the largest logit
-    bound of their token.  Returns the oracle's (idx, counts, offsets, perm)."""
+    """Indices and plan bit-exact; logits within the per-logit bound (and the
+    worst-case ceiling); weights within twice the largest logit bound of
+    their token.  Returns the oracle's (idx, counts, offsets, perm)."""
     T, k, E = cfg.T, cfg.k, cfg.E
     lg = oracle.router(inp["x"], inp["w_router"], inp["router_bias"], tokens=tokens)
     o_idx, o_w = oracle.topk_softmax(lg, k)
@@ -100,7 +118,7 @@ def check_routing(cfg: MoEConfig, inp: dict, res: dict, tokens=None):
     sel = slice(None) if tokens is None else np.asarray(tokens)
     assert np.array_equal(g_idx[sel], o_idx), "routing indices differ"
     x_sel = inp["x"] if tokens is None else inp["x"][torch.as_tensor(np.asarray(tokens))]
-    scale = logit_scale(x_sel, inp["w_router"], inp["router_bias"])
+    scale = logit_scale(x_sel, inp["w_router"], inp["router_bias"], router_chain_length(cfg))
     errs = [np.abs(res["logits"].numpy()[sel] - lg)]
     if "logits_split" in res:
         errs.append(np.abs(res["logits_split"].numpy()[sel] - lg))
@@ -109,14 +127,10 @@ def check_routing(cfg: MoEConfig, inp: dict, res: dict, tokens=None):
     ceiling = logit_tol(cfg.H, lg)
     assert lerr <= ceiling, f"logit error {lerr:.3e} > worst-case {ceiling:.3e}"
     werr_tok = np.abs(g_w[sel] - o_w).max(axis=1)
-    c = C_LOGIT if C_LOGIT is not None else 1.0
-    wtol_tok = 2.0 * c * scale.max(axis=1) + 1e-7
+    wtol_tok = 2.0 * C_LOGIT * scale.max(axis=1) + 1e-7
     wratio = float((werr_tok / wtol_tok).max())
-    if C_LOGIT is not None:
-        assert ratio <= C_LOGIT, f"logit error {ratio:.3f} x the per-logit scale > {C_LOGIT}"
-        assert wratio <= 1.0, f"routing weight error {wratio:.3f} x its bound"
-    else:
-        assert float(werr_tok.max()) <= 2 * ceiling, "routing weight error above 2x ceiling"
+    assert ratio <= C_LOGIT, f"logit error {ratio:.3f} x the per-logit bound"
+    assert wratio <= 1.0, f"routing weight error {wratio:.3f} x its bound"
     print(f"[{cfg.name}] logit error {lerr:.2e} = {ratio:.3f} x scale "
           f"(scale max {float(scale.max()):.2e}), weight error "
           f"{float(werr_tok.max()):.2e} = {wratio:.3f} x bound")
