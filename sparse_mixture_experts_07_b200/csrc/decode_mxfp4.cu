@@ -11,7 +11,8 @@
 // Storage: q [rows, K/2] bytes, element 2j of a row in the low nibble of byte
 // j, element 2j+1 in the high nibble; s [rows, K/32] bytes.
 //
-// Work unit: (expert group, chunk of 8*NT of its rows, 16 weight rows).  The
+// Work unit: (expert group, chunk of 8*NT of its rows, 16 weight rows), NT = 1
+// for batches of up to 8 tokens and 2 above.  The
 // MMAs are mma.sync m16n8k16 with weight rows as M and the chunk's token rows
 // as NT tiles of N = 8.  Per CTA, a ring of shared-memory stages, each holding
 // 512 weights of every row of the unit (gate and up rows for GEMM 1):
@@ -107,10 +108,12 @@ __global__ void __launch_bounds__(mx::PREP_THREADS) rows_to_f16_kernel(
     if (threadIdx.x == 0) exps[r] = p;
 }
 
+// Not volatile: a pure function of its operands, so the compiler may
+// interleave the MMAs of independent blocks.
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                               uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1,
                                               const float (&c)[4]) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
@@ -216,7 +219,7 @@ struct MxGeo {
     static constexpr int S_BYTES = R * mx::SWORDS * 4;             // scale words per stage
     static constexpr int NF = MAT * NT * 4;                        // accumulators per lane
     static constexpr int CONV_FLOATS = mx::CONSUMERS * R * mx::BPW;
-    static constexpr int RED_FLOATS = mx::CONSUMERS * NF * 32;
+    static constexpr int RED_FLOATS = 2 * mx::CONSUMERS * NF * 32;   // double-buffered
     static constexpr int FIXED = 1024 + 4 * (CONV_FLOATS + RED_FLOATS);
     static constexpr int STAGES_FIT = (mx::CTA_SMEM - FIXED) / (Q_BYTES + S_BYTES + 16);
     static constexpr int STAGES = STAGES_FIT < 3 ? 3 : (STAGES_FIT > 16 ? 16 : STAGES_FIT);
@@ -224,7 +227,8 @@ struct MxGeo {
 };
 
 // CTAs per SM the register budget is sized for: three with one n-tile, two
-// with four (their 32 accumulators per lane need more than 128 registers).
+// with more (their accumulators and prefetched fragments need more than 128
+// registers a thread).
 template <int NT>
 struct MxOccupancy {
     static constexpr int CTAS = NT == 1 ? 3 : 2;
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(mx::THREADS, MxOccupancy<NT>::CTAS) decode_mx_
     uint64_t* full = reinterpret_cast<uint64_t*>(s_ring + G::STAGES * G::S_BYTES);
     uint64_t* empty = full + G::STAGES;
     float* conv = reinterpret_cast<float*>(empty + G::STAGES);   // [CONSUMERS][R][BPW]
-    float* red = conv + G::CONV_FLOATS;                          // [CONSUMERS][NF][32]
+    float* red = conv + G::CONV_FLOATS;                          // [2][CONSUMERS][NF][32]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t deadline = global_ns() + timeout_ns;
 
@@ -387,20 +391,23 @@ __global__ void __launch_bounds__(mx::THREADS, MxOccupancy<NT>::CTAS) decode_mx_
         float acc[G::NF];
 #pragma unroll
         for (int j = 0; j < G::NF; ++j) acc[j] = 0.f;
-        // NT = 1: this warp's activation fragments, loaded one stage ahead
-        uint4 bv[BPW];
-        if (NT == 1) {
+        // this warp's activation fragments (BPW blocks x NT tiles), loaded one
+        // stage ahead of their use
+        uint4 bv[BPW][NT];
 #pragma unroll
-            for (int i = 0; i < BPW; ++i) bv[i] = ldg_v4(brow[0] + (cw * BPW + i) * 32);
-        }
+        for (int i = 0; i < BPW; ++i)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) bv[i][nt] = ldg_v4(brow[nt] + (cw * BPW + i) * 32);
         for (int st = 0; st < nst; ++st, ++f) {
             const int slot = f % G::STAGES;
             const uint32_t ph = static_cast<uint32_t>(f / G::STAGES) & 1u;
-            uint4 bn[BPW];
-            if (NT == 1 && st + 1 < nst) {
+            uint4 bn[BPW][NT];
+            if (st + 1 < nst) {
 #pragma unroll
                 for (int i = 0; i < BPW; ++i)
-                    bn[i] = ldg_v4(brow[0] + ((st + 1) * BPS + cw * BPW + i) * 32);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        bn[i][nt] = ldg_v4(brow[nt] + ((st + 1) * BPS + cw * BPW + i) * 32);
             }
             if (ok && !mbar_wait(&full[slot], ph, deadline)) ok = false;
             // this warp's blocks' scales as floats, once per stage (lane = row)
@@ -448,7 +455,7 @@ __global__ void __launch_bounds__(mx::THREADS, MxOccupancy<NT>::CTAS) decode_mx_
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const uint4 xv = NT == 1 ? bv[i] : ldg_v4(brow[nt] + (st * BPS + jj) * 32);
+                    const uint4 xv = bv[i][nt];
                     float d[4];
                     mx_block_mma(d, a, b, xv);
                     float* ag = acc + nt * 4;
@@ -469,22 +476,29 @@ __global__ void __launch_bounds__(mx::THREADS, MxOccupancy<NT>::CTAS) decode_mx_
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
-            if (NT == 1) {
+            if (st + 1 < nst) {
 #pragma unroll
-                for (int i = 0; i < BPW; ++i) bv[i] = bn[i];
+                for (int i = 0; i < BPW; ++i)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) bv[i][nt] = bn[i][nt];
             }
         }
-        // partial sums of the consumer warps meet in shared memory
+        // partial sums of the consumer warps meet in shared memory, in one of
+        // two buffers by unit parity: warp 1 reduces unit ui's buffer after the
+        // barrier while the other warps go on to unit ui + 1, whose barrier they
+        // cannot pass before warp 1 has finished with this buffer
+        float* rb = red + (ui & 1) * (CONSUMERS * G::NF * 32);
 #pragma unroll
-        for (int j = 0; j < G::NF; ++j) red[(cw * G::NF + j) * 32 + lane] = acc[j];
+        for (int j = 0; j < G::NF; ++j) rb[(cw * G::NF + j) * 32 + lane] = acc[j];
         if (!ok) fail_sh = 1;
         asm volatile("bar.sync 1, %0;" ::"r"(32 * CONSUMERS) : "memory");
+        const bool failed = fail_sh != 0;
         if (cw == 0) {
 #pragma unroll
             for (int j = 0; j < G::NF; ++j) {
                 float v = 0.f;
 #pragma unroll
-                for (int w = 0; w < CONSUMERS; ++w) v += red[(w * G::NF + j) * 32 + lane];
+                for (int w = 0; w < CONSUMERS; ++w) v += rb[(w * G::NF + j) * 32 + lane];
                 acc[j] = v;
             }
             // acc[nt*4 + 0..1]: weight row g, tokens 2q, 2q+1 of n-tile nt;
@@ -508,8 +522,7 @@ __global__ void __launch_bounds__(mx::THREADS, MxOccupancy<NT>::CTAS) decode_mx_
                     }
                 }
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(32 * CONSUMERS) : "memory");
-        if (fail_sh) break;
+        if (failed) break;
     }
     if (cw == 0 && lane == 0 && !ok) raise_error(p.err_flag, MOE_ERR_TIMEOUT);
 }
@@ -590,15 +603,17 @@ cudaError_t launch_ffn_decode_mxfp4(const moe_shape& s, const void* x, const int
         static_cast<const __nv_bfloat16*>(x), static_cast<__half*>(x16), xexp, s.H, p.ldx);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // one n-tile of 8 token rows covers every group of a batch of <= 8 tokens
+    // one n-tile of 8 token rows covers every group of a batch of <= 8 tokens;
+    // above, chunks of 16 rows (two tiles): a group of more rows streams its
+    // weights once per chunk, which at T <= 64 is rare (2 T / E rows on average)
     const bool small = s.T <= 8;
-    e = small ? launch_mx<0, 1>(map_gu, p, num_sms, st) : launch_mx<0, 4>(map_gu, p, num_sms, st);
+    e = small ? launch_mx<0, 1>(map_gu, p, num_sms, st) : launch_mx<0, 2>(map_gu, p, num_sms, st);
     if (e != cudaSuccess) return e;
     rows_to_f16_kernel<<<static_cast<unsigned>(s.T * s.k), mx::PREP_THREADS, 0, st>>>(
         static_cast<const __nv_bfloat16*>(h), static_cast<__half*>(h16), hexp, s.I, p.ldh);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return small ? launch_mx<1, 1>(map_dn, p, num_sms, st) : launch_mx<1, 4>(map_dn, p, num_sms, st);
+    return small ? launch_mx<1, 1>(map_dn, p, num_sms, st) : launch_mx<1, 2>(map_dn, p, num_sms, st);
 }
 
 }  // namespace moe
