@@ -38,8 +38,8 @@ L2_BYTES = 126 * 1024 * 1024
 # kernels, from one ncu capture, keyed by workload; valid only while the GEMM
 # source is unchanged (sha256 of the file, first 16 hex digits).
 TRAFFIC = {
-    # profiles/grouped_gemm_pair_mixtral.md: gather 0.053 + GEMM 1 3.410 + GEMM 2 1.687 GB
-    "mixtral": {"bytes": 5.149e9, "file": "gemm_sm100_pair.cu", "sha": "1ef98e621b42032d"},
+    # profiles/traffic_mixtral.md: gather 0.053 + GEMM 1 2.527 + GEMM 2 1.473 GB
+    "mixtral": {"bytes": 4.053e9, "file": "gemm_sm100_pair.cu", "sha": "1d599c5a5dbfdc6f"},
 }
 
 
