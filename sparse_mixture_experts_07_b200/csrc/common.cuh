@@ -126,12 +126,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: spins until the phase with `parity` completes, or until
-// `deadline_ns` (globaltimer) passes; returns false on timeout.
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended (it issues nothing) until the phase completes or about hint_ns
+// nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: until the phase with `parity` completes, or until
+// `deadline_ns` (globaltimer) passes; returns false on timeout.  Waiting
+// threads are suspended between checks (at most about 20 us each), so warps
+// that wait do not take issue slots from the warps that work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline_ns) {
-    uint32_t n = 0;
-    while (!mbar_try_wait(bar, parity)) {
-        if ((++n & 1023u) == 0 && global_ns() > deadline_ns) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
+        if (global_ns() > deadline_ns) return false;
     }
     return true;
 }
