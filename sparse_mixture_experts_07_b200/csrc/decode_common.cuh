@@ -58,6 +58,43 @@ __device__ __forceinline__ int find_active(const ActiveGroups& a, int unit) {
     return lo;
 }
 
+// Expert groups with rows, each with ceil(rows / chunk_rows) chunks of
+// units_per_chunk work units (the MXFP4 decode kernels).  Built by one thread
+// from a.offs, which stage_offsets filled.
+struct MxUnits {
+    int n;
+    int total_units;
+    int gid[kMaxExperts];
+    int unit_start[kMaxExperts + 1];
+    int32_t offs[kMaxExperts + 1];
+};
+
+__device__ __forceinline__ void build_mx_units(MxUnits& a, int E, int chunk_rows,
+                                               int units_per_chunk) {
+    int n = 0, acc = 0;
+    for (int g = 0; g < E; ++g) {
+        const int rows = a.offs[g + 1] - a.offs[g];
+        if (rows <= 0) continue;
+        a.gid[n] = g;
+        a.unit_start[n] = acc;
+        acc += ((rows + chunk_rows - 1) / chunk_rows) * units_per_chunk;
+        ++n;
+    }
+    a.unit_start[n] = acc;
+    a.n = n;
+    a.total_units = acc;
+}
+
+__device__ __forceinline__ int find_mx_unit(const MxUnits& a, int unit) {
+    int lo = 0, hi = a.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.unit_start[mid] <= unit) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
 // Not volatile: a pure function of its operands, so the compiler may
 // interleave independent MMA chains.
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,

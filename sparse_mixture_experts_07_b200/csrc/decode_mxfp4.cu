@@ -173,41 +173,6 @@ __device__ __forceinline__ void mx_block_mma(float (&d)[4], const uint32_t (&a)[
     mma_f16_16816(d, a[2], b[2], a[3], b[3], xv.z, xv.w, d);
 }
 
-// Expert groups with rows, each with ceil(rows / (8 NT)) chunks x N/16 units.
-struct MxUnits {
-    int n;
-    int total_units;
-    int gid[kMaxExperts];
-    int unit_start[kMaxExperts + 1];
-    int32_t offs[kMaxExperts + 1];
-};
-
-__device__ __forceinline__ void build_mx_units(MxUnits& a, int E, int chunk_rows,
-                                               int units_per_chunk) {
-    int n = 0, acc = 0;
-    for (int g = 0; g < E; ++g) {
-        const int rows = a.offs[g + 1] - a.offs[g];
-        if (rows <= 0) continue;
-        a.gid[n] = g;
-        a.unit_start[n] = acc;
-        acc += ((rows + chunk_rows - 1) / chunk_rows) * units_per_chunk;
-        ++n;
-    }
-    a.unit_start[n] = acc;
-    a.n = n;
-    a.total_units = acc;
-}
-
-__device__ __forceinline__ int find_mx_unit(const MxUnits& a, int unit) {
-    int lo = 0, hi = a.n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a.unit_start[mid] <= unit) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
 // Stage geometry.  KIND 0: gate_up (K = H, output rows I; a stage holds NB
 // boxes of the unit's 16 gate rows and NB of the matching 16 up rows).
 // KIND 1: down (K = I, output rows H; NB boxes of 16 rows).

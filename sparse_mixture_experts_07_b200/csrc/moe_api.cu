@@ -15,6 +15,8 @@ cudaError_t launch_route_tc_split(const moe_shape&, const void*, const void*, co
                                   int32_t*, float*, int32_t*, int, cudaStream_t);
 cudaError_t launch_route_small(const moe_shape&, const void*, const float*, const float*, float*,
                                int32_t*, float*, cudaStream_t);
+cudaError_t launch_route_cluster(const moe_shape&, const void*, const float*, const float*, float*,
+                               int32_t*, float*, cudaStream_t);
 size_t permute_workspace_bytes(const moe_shape&);
 cudaError_t launch_permute(const moe_shape&, const int32_t*, int32_t*, int32_t*, int32_t*,
                            int32_t*, int32_t*, void*, cudaStream_t);
@@ -38,6 +40,14 @@ cudaError_t launch_ffn_decode_mxfp4(const moe_shape&, const void*, const int32_t
                                     int32_t*, void*, int32_t*, int, cudaStream_t);
 cudaError_t launch_combine(const moe_shape&, const void*, const int32_t*, void*, cudaStream_t);
 int mx_padded_cols(int K);
+bool mx_tc_supported(const moe_shape&, const void*, const void*);
+int64_t mx_tc_plane_rows(int64_t slots);
+int64_t mx_tc_part_floats(int64_t slots, int H, int I);
+cudaError_t launch_ffn_decode_mxfp4_tc(const moe_shape&, const void*, const int32_t*,
+                                       const int32_t*, const float*, const uint8_t*,
+                                       const uint8_t*, const uint8_t*, const uint8_t*, uint8_t*,
+                                       uint8_t*, uint8_t*, uint8_t*, float*, int32_t*, void*,
+                                       int32_t*, int, cudaStream_t);
 cudaError_t launch_combine_experts(const moe_shape&, int, int, int, const void*, const int32_t*,
                                    const int32_t*, float*, int, cudaStream_t);
 cudaError_t launch_cast_f32(const moe_shape&, const float*, void*, int, cudaStream_t);
@@ -106,6 +116,7 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 struct Workspace {
     size_t permute_off, h_routed_off, h_shared_off, x_perm_off, inv_off;
     size_t mx_x16_off, mx_xexp_off, mx_h16_off, mx_hexp_off;   // MXFP4 decode (T <= 64)
+    size_t mx_xq_off, mx_xsf_off, mx_hq_off, mx_hsf_off, mx_part_off, mx_ctl_off;
     size_t total;
 };
 
@@ -134,6 +145,23 @@ Workspace layout(const moe_shape& s) {
         off += align_up(static_cast<size_t>(Tk) * moe::mx_padded_cols(s.I) * 2);
         w.mx_hexp_off = off;
         off += align_up(static_cast<size_t>(Tk) * 4);
+        if (s.H % 128 == 0 && s.I % 128 == 0) {
+            // block-scaled tensor-core path: E4M3 hi/lo planes of x and h with
+            // their exponents, the split partials, and the split count
+            const size_t SP = static_cast<size_t>(moe::mx_tc_plane_rows(Tk));
+            w.mx_xq_off = off;
+            off += align_up(2 * SP * s.H);
+            w.mx_xsf_off = off;
+            off += align_up(2 * SP * (s.H / 32));
+            w.mx_hq_off = off;
+            off += align_up(2 * SP * s.I);
+            w.mx_hsf_off = off;
+            off += align_up(2 * SP * (s.I / 32));
+            w.mx_part_off = off;
+            off += align_up(static_cast<size_t>(moe::mx_tc_part_floats(Tk, s.H, s.I)) * 4);
+            w.mx_ctl_off = off;
+            off += align_up(16);
+        }
     }
     w.total = off;
     return w;
@@ -172,10 +200,16 @@ moe_status moe_route(const moe_shape* shape, const void* x, const float* w_route
     if (shape->T == 0) return MOE_OK;
     if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    // few tokens: one CTA per token; many tokens, bf16: tensor cores; else CUDA cores
-    if (shape->T <= 256 && shape->H <= 32768 && aligned16(w_router))
+    // few tokens: a cluster per 16 tokens splitting the hidden dimension (one
+    // CTA per token where its shared memory does not fit); many tokens, bf16:
+    // tensor cores; else CUDA cores
+    if (shape->T <= 256 && shape->H <= 32768 && aligned16(w_router)) {
+        const cudaError_t e = moe::launch_route_cluster(*shape, x, w_router, router_bias, logits,
+                                                        topk_idx, topk_w, cs);
+        if (e != cudaErrorNotSupported) return cuda_status(e);
         return cuda_status(moe::launch_route_small(*shape, x, w_router, router_bias, logits,
                                                    topk_idx, topk_w, cs));
+    }
     if (shape->dtype == MOE_BF16 && shape->E <= 64 && aligned16(x) && aligned16(w_router))
         return cuda_status(moe::launch_route_tc(*shape, x, w_router, router_bias, logits,
                                                 topk_idx, topk_w, err_flag, cs));
@@ -588,6 +622,13 @@ moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x, const int32_
     if ((reinterpret_cast<uintptr_t>(gate_up_s) & 3u) || (reinterpret_cast<uintptr_t>(down_s) & 3u))
         return MOE_ERR_UNSUPPORTED;
     char* ws = static_cast<char*>(workspace);
+    if (moe::mx_tc_supported(s, gate_up_q, down_q))
+        return cuda_status(moe::launch_ffn_decode_mxfp4_tc(
+            s, x, offsets, perm, topk_w, gate_up_q, gate_up_s, down_q, down_s,
+            reinterpret_cast<uint8_t*>(ws + w.mx_xq_off), reinterpret_cast<uint8_t*>(ws + w.mx_xsf_off),
+            reinterpret_cast<uint8_t*>(ws + w.mx_hq_off), reinterpret_cast<uint8_t*>(ws + w.mx_hsf_off),
+            reinterpret_cast<float*>(ws + w.mx_part_off), reinterpret_cast<int32_t*>(ws + w.mx_ctl_off),
+            y_slots, err_flag, num_sms(), static_cast<cudaStream_t>(stream)));
     return cuda_status(moe::launch_ffn_decode_mxfp4(
         s, x, offsets, perm, topk_w, gate_up_q, gate_up_s, down_q, down_s, ws + w.h_routed_off,
         ws + w.mx_x16_off, reinterpret_cast<int32_t*>(ws + w.mx_xexp_off), ws + w.mx_h16_off,

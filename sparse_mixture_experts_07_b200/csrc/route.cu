@@ -133,6 +133,51 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     }
 }
 
+// One warp: writes the token's logits lg[0..E) (if `logits`), then selects the
+// top k (k rounds of a warp arg-max, ties to the lower expert index) and
+// writes their indices and the softmax over the selected logits.
+__device__ __forceinline__ void select_topk_warp(const float* lg, int E, int k, int64_t tok,
+                                                 float* __restrict__ logits,
+                                                 int32_t* __restrict__ topk_idx,
+                                                 float* __restrict__ topk_w) {
+    const int lane = threadIdx.x & 31;
+    if (logits)
+        for (int e = lane; e < E; e += 32) logits[tok * E + e] = lg[e];
+    float sel_v[kMaxK];
+    int sel_e[kMaxK];
+    for (int r = 0; r < k; ++r) {
+        float best = -INFINITY;
+        int best_e = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            bool taken = false;
+            for (int q = 0; q < r; ++q) taken |= (sel_e[q] == e);
+            if (!taken && (lg[e] > best || best_e == 0x7fffffff)) {
+                best = lg[e];
+                best_e = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
+            if (ov > best || (ov == best && oe < best_e)) {
+                best = ov;
+                best_e = oe;
+            }
+        }
+        sel_v[r] = best;
+        sel_e[r] = best_e;
+    }
+    if (lane == 0) {
+        float den = 0.f;
+        for (int r = 0; r < k; ++r) den += expf(sel_v[r] - sel_v[0]);
+        for (int r = 0; r < k; ++r) {
+            topk_idx[tok * k + r] = sel_e[r];
+            topk_w[tok * k + r] = expf(sel_v[r] - sel_v[0]) / den;
+        }
+    }
+}
+
 // Few tokens (decode): one CTA per token, 8 warps over the experts.  The token
 // row is staged in shared memory as float32; warp w computes the logits of
 // experts w, w+8, ...: each lane reads 4 consecutive weights per step (16-byte
@@ -187,41 +232,128 @@ __global__ void __launch_bounds__(256) route_small_kernel(
     }
     __syncthreads();
     if (warp != 0) return;
-    if (logits)
-        for (int e = lane; e < E; e += 32) logits[tok * E + e] = lg[e];
-    float sel_v[kMaxK];
-    int sel_e[kMaxK];
-    for (int r = 0; r < k; ++r) {
-        float best = -INFINITY;
-        int best_e = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            bool taken = false;
-            for (int q = 0; q < r; ++q) taken |= (sel_e[q] == e);
-            if (!taken && (lg[e] > best || best_e == 0x7fffffff)) {
-                best = lg[e];
-                best_e = e;
+    select_topk_warp(lg, E, k, tok, logits, topk_idx, topk_w);
+}
+
+// Decode batches (at most kRouteClusterTokens tokens per cluster): a cluster
+// of kRouteCluster CTAs per block of tokens, CTA r owning hidden columns
+// [r HS, (r+1) HS).  Each CTA stages its slice of the tokens' rows in shared
+// memory and computes the partial logits of every (token, expert) over its
+// slice (warp w: experts w, w+8, ...; 16-byte loads of the router weights,
+// lane partials summed by a butterfly).  After a cluster barrier, CTA 0 adds
+// the kRouteCluster partials of each logit in rank order through distributed
+// shared memory, adds the bias and selects as above; a second barrier keeps
+// the other CTAs' shared memory alive until it has read it.  The router
+// weights are read once per token block, spread over kRouteCluster SMs.
+constexpr int kRouteCluster = 8;
+constexpr int kRouteClusterTokens = 16;
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) route_cluster_kernel(
+    const T* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
+    float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int64_t n_tokens, int H, int E, int k, int HS) {
+    extern __shared__ float4 smem_f4[];
+    float* part = reinterpret_cast<float*>(smem_f4);              // [TB][E] partial logits
+    float* xs = part + ((kRouteClusterTokens * E + 3) & ~3);      // [TB][HS]
+    const uint32_t rank = cluster_ctarank();
+    const int64_t tok0 = static_cast<int64_t>(cluster_id_x()) * kRouteClusterTokens;
+    const int tb = static_cast<int>(n_tokens - tok0 < kRouteClusterTokens ? n_tokens - tok0
+                                                                          : kRouteClusterTokens);
+    const int h0 = static_cast<int>(rank) * HS;
+    const int hs = H - h0 < HS ? (H - h0 > 0 ? H - h0 : 0) : HS;   // columns of this slice
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < tb * HS; i += 256) {
+        const int t = i / HS, h = i - t * HS;
+        xs[i] = h < hs ? ElemIO<T>::load(x, (tok0 + t) * H + h0 + h) : 0.f;
+    }
+    __syncthreads();
+    // HS is a multiple of 4 and the slice starts on a 16-byte boundary of
+    // each weight row when H % 4 == 0 (the launcher's condition)
+    const int n4 = hs >> 2;
+    for (int e = warp; e < E; e += 8) {
+        const float4* w = reinterpret_cast<const float4*>(wr + static_cast<int64_t>(e) * H + h0);
+        for (int t = 0; t < tb; ++t) {
+            const float4* xv = reinterpret_cast<const float4*>(xs + t * HS);
+            float acc = 0.f;
+            for (int i = lane; i < n4; i += 32) {
+                const float4 a = __ldg(w + i);
+                const float4 b = xv[i];
+                acc = fmaf(a.x, b.x, acc);
+                acc = fmaf(a.y, b.y, acc);
+                acc = fmaf(a.z, b.z, acc);
+                acc = fmaf(a.w, b.w, acc);
             }
-        }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
-            if (ov > best || (ov == best && oe < best_e)) {
-                best = ov;
-                best_e = oe;
-            }
-        }
-        sel_v[r] = best;
-        sel_e[r] = best_e;
-    }
-    if (lane == 0) {
-        float den = 0.f;
-        for (int r = 0; r < k; ++r) den += expf(sel_v[r] - sel_v[0]);
-        for (int r = 0; r < k; ++r) {
-            topk_idx[tok * k + r] = sel_e[r];
-            topk_w[tok * k + r] = expf(sel_v[r] - sel_v[0]) / den;
+            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) part[t * E + e] = acc;
         }
     }
+    cluster_sync();
+    if (rank == 0) {
+        // logits = sum of the ranks' partials in rank order (+ bias), kept in
+        // this CTA's xs (no longer needed)
+        float* lg = xs;
+        const uint32_t base = smem_u32(part);
+        for (int i = tid; i < tb * E; i += 256) {
+            float v = 0.f;
+            for (int r = 0; r < kRouteCluster; ++r)
+                v += ld_shared_cluster_f32(mapa_shared(base + 4u * static_cast<uint32_t>(i),
+                                                       static_cast<uint32_t>(r)));
+            lg[i] = v + (bias ? bias[i % E] : 0.f);
+        }
+        __syncthreads();
+        for (int t = warp; t < tb; t += 8)
+            select_topk_warp(lg + t * E, E, k, tok0 + t, logits, topk_idx, topk_w);
+    }
+    cluster_sync();
+}
+
+// The cluster kernel when its shared memory fits (decode batches); returns
+// cudaErrorNotSupported otherwise so that the caller takes route_small.
+cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float* wr,
+                                 const float* bias, float* logits, int32_t* idx, float* w,
+                                 cudaStream_t st) {
+    if (s.H % 4 != 0 || s.T > 64 * kRouteClusterTokens) return cudaErrorNotSupported;
+    const int HS = ((s.H + kRouteCluster - 1) / kRouteCluster + 3) & ~3;
+    const size_t smem = sizeof(float) * (((kRouteClusterTokens * s.E + 3) & ~3) +
+                                         static_cast<size_t>(kRouteClusterTokens) * HS);
+    if (smem > 96 * 1024 || static_cast<size_t>(kRouteClusterTokens) * s.E >
+                                static_cast<size_t>(kRouteClusterTokens) * HS)
+        return cudaErrorNotSupported;
+    const int blocks = static_cast<int>((s.T + kRouteClusterTokens - 1) / kRouteClusterTokens);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks * kRouteCluster));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kRouteCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (s.dtype == MOE_BF16) {
+        auto kern = route_cluster_kernel<__nv_bfloat16>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(x), wr, bias, logits,
+                                  idx, w, static_cast<int64_t>(s.T), s.H, s.E, s.k, HS);
+    }
+    auto kern = route_cluster_kernel<float>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const float*>(x), wr, bias, logits, idx, w,
+                              static_cast<int64_t>(s.T), s.H, s.E, s.k, HS);
 }
 
 cudaError_t launch_route_small(const moe_shape& s, const void* x, const float* wr,
