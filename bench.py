@@ -287,7 +287,7 @@ def roofline_of(cfg, counts, fwd_ms, region_s, mxfp4, peaks, traffic=None) -> di
         return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                 "algorithmic_bytes": algo,
-                "kernel": "moe_forward_mxfp4 (f16 prep + MXFP4 expert FFN launches)"
+                "kernel": "moe_forward_mxfp4 (activation prep, MXFP4 expert GEMMs and their epilogues)"
                           if mxfp4 else "moe_forward (expert FFN launches)",
                 "peak_kind": f"{peaks['source']} HBM copy"}
     flops = 2.0 * cfg.T * (3 * cfg.k * cfg.H * cfg.I + 3 * cfg.n_shared * cfg.I_shared * cfg.H)

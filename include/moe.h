@@ -256,12 +256,19 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const int3
  *   gate_up_s [E, 2I, H/32] uint8 E8M0 scale of each block of 32 weights
  *   down_q    [E, H, I/2]   uint8, same packing;  down_s [E, H, I/32] uint8
  * Other arguments, outputs and workspace as moe_forward (y_slots holds the
- * T*k routed rows).  Supported: bf16 x, 1 <= T <= 8, no shared experts, H and
- * I multiples of 32; otherwise MOE_ERR_UNSUPPORTED.  The products run in f16
- * with float32 accumulation: each activation row (x, then h) is scaled by a
- * power of two that puts its largest magnitude in [2^14, 2^15) and rounded to
- * f16; the scaling is undone in float32.  Weights must stay below 2^128 in
- * magnitude (scale codes up to 252). */
+ * T*k routed rows).  Supported: bf16 x, 1 <= T <= 64, no shared experts, H
+ * and I multiples of 32, the scale arrays 4-byte aligned; otherwise
+ * MOE_ERR_UNSUPPORTED.  Two kernels, chosen by shape:
+ *   - H and I multiples of 128 and the code arrays 32-byte aligned: the
+ *     block-scaled tensor-core MMA (E2M1 weights x E4M3 activations, E8M0
+ *     scales on both).  Each bf16 activation (x, then h rounded to bf16) is
+ *     split per block of 32 into two E4M3 parts under E8M0 exponents, which
+ *     reproduce it exactly except for elements below about 2^-13 of their
+ *     block's largest magnitude; float32 accumulation.
+ *   - otherwise: f16 MMAs with float32 accumulation; each activation row is
+ *     scaled by a power of two that puts its largest magnitude in
+ *     [2^14, 2^15) and rounded to f16; the scaling is undone in float32.
+ * Weights must stay below 2^128 in magnitude (scale codes up to 252). */
 MOE_API moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x,
                                      const int32_t* offsets, const int32_t* perm,
                                      const float* topk_w, const uint8_t* gate_up_q,

@@ -248,20 +248,28 @@ __global__ void __launch_bounds__(256) route_small_kernel(
 constexpr int kRouteCluster = 8;
 constexpr int kRouteClusterTokens = 16;
 
+// Volatile (kept in order with the cluster barriers) but without a memory
+// clobber, so that a thread's loads are all in flight before their first use.
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
+}
+
+__device__ __forceinline__ void cp_async16_route(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256) route_cluster_kernel(
     const T* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
     float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    int64_t n_tokens, int H, int E, int k, int HS) {
+    int64_t n_tokens, int H, int E, int k, int HS, int stage_w) {
     extern __shared__ float4 smem_f4[];
     float* part = reinterpret_cast<float*>(smem_f4);              // [TB][E] partial logits
     float* xs = part + ((kRouteClusterTokens * E + 3) & ~3);      // [TB][HS]
+    float* ws = xs + kRouteClusterTokens * HS;                    // [E][HS] if stage_w
     const uint32_t rank = cluster_ctarank();
     const int64_t tok0 = static_cast<int64_t>(cluster_id_x()) * kRouteClusterTokens;
     const int tb = static_cast<int>(n_tokens - tok0 < kRouteClusterTokens ? n_tokens - tok0
@@ -269,21 +277,34 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(
     const int h0 = static_cast<int>(rank) * HS;
     const int hs = H - h0 < HS ? (H - h0 > 0 ? H - h0 : 0) : HS;   // columns of this slice
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // HS is a multiple of 4 and the slice starts on a 16-byte boundary of
+    // each weight row when H % 4 == 0 (the launcher's condition)
+    const int n4 = hs >> 2;
+    if (stage_w) {
+        // the slice of every router row, all in flight at once (one memory
+        // latency instead of one per expert a warp handles)
+        const int q = HS >> 2;
+        for (int i = tid; i < E * q; i += 256) {
+            const int e = i / q, c = i - e * q;
+            if (c < n4) cp_async16_route(ws + e * HS + 4 * c, wr + static_cast<int64_t>(e) * H + h0 + 4 * c);
+        }
+    }
     for (int i = tid; i < tb * HS; i += 256) {
         const int t = i / HS, h = i - t * HS;
         xs[i] = h < hs ? ElemIO<T>::load(x, (tok0 + t) * H + h0 + h) : 0.f;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    // HS is a multiple of 4 and the slice starts on a 16-byte boundary of
-    // each weight row when H % 4 == 0 (the launcher's condition)
-    const int n4 = hs >> 2;
     for (int e = warp; e < E; e += 8) {
-        const float4* w = reinterpret_cast<const float4*>(wr + static_cast<int64_t>(e) * H + h0);
+        const float4* wg = reinterpret_cast<const float4*>(wr + static_cast<int64_t>(e) * H + h0);
+        // (points into xs when the slice is not staged, so that even a
+        // speculated load stays inside the allocation)
+        const float4* wsv = reinterpret_cast<const float4*>(stage_w ? ws + e * HS : xs);
         for (int t = 0; t < tb; ++t) {
             const float4* xv = reinterpret_cast<const float4*>(xs + t * HS);
             float acc = 0.f;
             for (int i = lane; i < n4; i += 32) {
-                const float4 a = __ldg(w + i);
+                const float4 a = stage_w ? wsv[i] : __ldg(wg + i);
                 const float4 b = xv[i];
                 acc = fmaf(a.x, b.x, acc);
                 acc = fmaf(a.y, b.y, acc);
@@ -302,10 +323,14 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(
         float* lg = xs;
         const uint32_t base = smem_u32(part);
         for (int i = tid; i < tb * E; i += 256) {
-            float v = 0.f;
+            float pv[kRouteCluster];
+#pragma unroll
             for (int r = 0; r < kRouteCluster; ++r)
-                v += ld_shared_cluster_f32(mapa_shared(base + 4u * static_cast<uint32_t>(i),
-                                                       static_cast<uint32_t>(r)));
+                pv[r] = ld_shared_cluster_f32(mapa_shared(base + 4u * static_cast<uint32_t>(i),
+                                                          static_cast<uint32_t>(r)));
+            float v = 0.f;
+#pragma unroll
+            for (int r = 0; r < kRouteCluster; ++r) v += pv[r];
             lg[i] = v + (bias ? bias[i % E] : 0.f);
         }
         __syncthreads();
@@ -322,11 +347,15 @@ cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float*
                                  cudaStream_t st) {
     if (s.H % 4 != 0 || s.T > 64 * kRouteClusterTokens) return cudaErrorNotSupported;
     const int HS = ((s.H + kRouteCluster - 1) / kRouteCluster + 3) & ~3;
-    const size_t smem = sizeof(float) * (((kRouteClusterTokens * s.E + 3) & ~3) +
-                                         static_cast<size_t>(kRouteClusterTokens) * HS);
+    size_t smem = sizeof(float) * (((kRouteClusterTokens * s.E + 3) & ~3) +
+                                   static_cast<size_t>(kRouteClusterTokens) * HS);
     if (smem > 96 * 1024 || static_cast<size_t>(kRouteClusterTokens) * s.E >
                                 static_cast<size_t>(kRouteClusterTokens) * HS)
         return cudaErrorNotSupported;
+    // stage the router slice in shared memory too when it fits
+    const size_t w_bytes = sizeof(float) * static_cast<size_t>(s.E) * HS;
+    const int stage_w = smem + w_bytes <= 160 * 1024 ? 1 : 0;
+    if (stage_w) smem += w_bytes;
     const int blocks = static_cast<int>((s.T + kRouteClusterTokens - 1) / kRouteClusterTokens);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks * kRouteCluster));
@@ -346,14 +375,14 @@ cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float*
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(x), wr, bias, logits,
-                                  idx, w, static_cast<int64_t>(s.T), s.H, s.E, s.k, HS);
+                                  idx, w, static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w);
     }
     auto kern = route_cluster_kernel<float>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const float*>(x), wr, bias, logits, idx, w,
-                              static_cast<int64_t>(s.T), s.H, s.E, s.k, HS);
+                              static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w);
 }
 
 cudaError_t launch_route_small(const moe_shape& s, const void* x, const float* wr,
