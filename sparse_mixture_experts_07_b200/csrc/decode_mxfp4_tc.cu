@@ -39,11 +39,14 @@
 // sums the splits in order (deterministic), then applies SiLU(gate) * up
 // (GEMM 1, which also quantises h for GEMM 2) or the routing weight (GEMM 2).
 //
-// One persistent CTA per SM, 192 threads:
-//   warp 0     producer: lane 0 issues the TMA boxes of a stage (two of 64
-//              weight rows, the hi and the lo activation box); all 32 lanes
-//              copy the stage's scale words with 4-byte cp.async and report
-//              them on the stage barrier with cp.async.mbarrier.arrive;
+// Persistent CTAs of 192 threads, two or three per SM (MxTcCfg): a
+// tcgen05 instruction costs its issuing thread a roughly fixed time whatever
+// its size, so the SM moves more bytes with more issuing threads.  Stages of
+// one K-group, weights as a 5D tensor-map box (the tile's two 64-row halves).
+//   warp 0     producer: lane 0 issues the TMA boxes of a stage (the weight
+//              tile, the hi and lo activation rows); all 32 lanes copy the
+//              stage's scale words with 4-byte cp.async and report them on
+//              the stage barrier with cp.async.mbarrier.arrive;
 //   warp 1     allocates tensor memory; one thread copies the stage's scale
 //              factors to tensor memory and issues its four MMAs;
 //   warps 2-5  epilogue: tcgen05.ld of their 32 lanes, hi + lo, fp32 partial
@@ -70,9 +73,19 @@ constexpr int PREP_THREADS = 256;          // 8 warps, one 32-block each
 constexpr int SMEM_BUDGET = 220 * 1024;
 }  // namespace mxtc
 
+// CTAs per SM (CPS) and K-groups per stage (KGS) by chunk size CH: as many
+// CTAs as the shared and tensor memory allow while each keeps at least three
+// stages (measured, PhiMoE shapes: CH = 8 at 3 CTAs 1.3x faster than 2 and
+// 1.15x faster than 4; CH = 16 at 2 CTAs 2 % faster than 3).
+template <int CH>
+struct MxTcCfg {
+    static constexpr int CPS = CH <= 8 ? 3 : 2;
+    static constexpr int KGS = 1;
+};
+
 // Stage geometry: KGS K-groups (KGS x 128 codes of each of the tile's 128
 // rows) per stage, CH activation rows per chunk.
-template <int CH, int KGS>
+template <int CH, int KGS, int CPS>
 struct TcGeo {
     static constexpr int N = 2 * CH;                       // MMA N: hi and lo rows
     static constexpr int A_SMEM = KGS * mxtc::A_KG_SMEM;   // [kg][128 rows][128 B]
@@ -82,19 +95,21 @@ struct TcGeo {
     static constexpr int SF_SMEM = 2 * KGS * mxtc::SF_ATOM;   // [kg] SFA atoms, then [kg] SFB
     static constexpr int STAGE = A_SMEM + B_SMEM + SF_SMEM;  // 1024-multiple
     static constexpr int TX = A_TX + B_SMEM;
-    static constexpr int STAGES = (mxtc::SMEM_BUDGET - 1024 - 256) / STAGE;
+    static constexpr int STAGES = (mxtc::SMEM_BUDGET / CPS - 1024 - 256) / STAGE;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + 256;
     // NACC accumulators per buffer, MMA kb of a K-group adding into
     // accumulator kb % NACC, so that consecutive MMAs do not wait for each
     // other's result; two buffers (the epilogue of one item overlaps the
     // next item's MMAs); two scale-factor slots used by alternate K-groups
-    static constexpr int NACC = N <= 32 ? 4 : 2;
+    // (as many as fit the tensor memory each of the CPS CTAs of an SM can hold)
+    static constexpr int TMEM_LIMIT = CPS == 1 ? 512 : (CPS == 2 ? 256 : 128);
+    static constexpr int NACC = 2 * 4 * N + 16 <= TMEM_LIMIT ? 4 : (2 * 2 * N + 16 <= TMEM_LIMIT ? 2 : 1);
     static constexpr int ACC_COLS = NACC * N;              // one buffer
     static constexpr int SF_COL = 2 * ACC_COLS;            // [2 slots][SFA 4 | SFB 4]
     static constexpr int COLS_USED = SF_COL + 16;
     static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64
                                    : COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
-    static_assert(COLS_USED <= 512, "tensor memory");
+    static_assert(TMEM_COLS <= TMEM_LIMIT, "tensor memory of CPS CTAs per SM");
     static_assert(STAGE % 1024 == 0, "stage must keep the 1024-byte swizzle alignment");
     static_assert(B_KG % 1024 == 0 && A_SMEM % 1024 == 0, "tiles must start on swizzle atoms");
     static_assert(STAGES >= 2 && 2 * STAGES + 5 <= 32, "stage count / barrier space");
@@ -234,11 +249,11 @@ __host__ __device__ inline int mx_tc_splits(int units, int grid, int n_kg, int k
 //   GEMM 2: R1 = 64, R2 = H/64: box rows (0..63, 2mt..2mt+1)
 // map_act: the E4M3 planes as a 4D tensor (128 bytes of a K-group, SP rows,
 // 2 planes, K/128 K-groups): box (CH rows, both planes, KGS K-groups).
-template <int KIND, int CH, int KGS>
-__global__ void __launch_bounds__(mxtc::THREADS, 1) decode_mx_tc_kernel(
+template <int KIND, int CH, int KGS, int CPS>
+__global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_act,
     const MxTcParams p) {
-    using G = TcGeo<CH, KGS>;
+    using G = TcGeo<CH, KGS, CPS>;
     using namespace mxtc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ MxUnits act;
@@ -640,19 +655,19 @@ bool mx_tc_supported(const moe_shape& s, const void* gu_q, const void* dn_q) {
            (reinterpret_cast<uintptr_t>(dn_q) & 31u) == 0;
 }
 
-template <int KIND, int CH, int KGS>
+template <int KIND, int CH, int KGS, int CPS>
 static cudaError_t launch_tc(const CUtensorMap& mw, const CUtensorMap& ma, const MxTcParams& p,
                              int num_sms, cudaStream_t st) {
-    using G = TcGeo<CH, KGS>;
-    auto kern = decode_mx_tc_kernel<KIND, CH, KGS>;
+    using G = TcGeo<CH, KGS, CPS>;
+    auto kern = decode_mx_tc_kernel<KIND, CH, KGS, CPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          G::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, mxtc::THREADS, G::SMEM_BYTES, st>>>(mw, ma, p);
+    kern<<<CPS * num_sms, mxtc::THREADS, G::SMEM_BYTES, st>>>(mw, ma, p);
     return cudaGetLastError();
 }
 
-template <int CH, int KGS>
+template <int CH, int KGS, int CPS>
 static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offsets,
                           const int32_t* perm, const float* topk_w, const uint8_t* gu_q,
                           const uint8_t* gu_s, const uint8_t* dn_q, const uint8_t* dn_s,
@@ -693,7 +708,7 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
     p.wrows = 2 * static_cast<int64_t>(s.I);
     p.n_out = 2 * s.I;
     p.mtiles = s.I / mxtc::HALF_ROWS;
-    e = launch_tc<0, CH, KGS>(map_gu, map_x, p, num_sms, st);
+    e = launch_tc<0, CH, KGS, CPS>(map_gu, map_x, p, num_sms, st);
     if (e != cudaSuccess) return e;
     mx_tc_swiglu_kernel<<<dim3((s.I / 32 + WPB - 1) / WPB, S), mxtc::PREP_THREADS, 0, st>>>(
         part, ctl, S, s.I, SP, hq, hsf);
@@ -706,7 +721,7 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
     p.wrows = s.H;
     p.n_out = s.H;
     p.mtiles = s.H / 128;
-    e = launch_tc<1, CH, KGS>(map_dn, map_h, p, num_sms, st);
+    e = launch_tc<1, CH, KGS, CPS>(map_dn, map_h, p, num_sms, st);
     if (e != cudaSuccess) return e;
     mx_tc_down_out_kernel<<<dim3((s.H + 255) / 256, S), 256, 0, st>>>(
         part, ctl, perm, topk_w, s.routed_scale, S, s.H, static_cast<__nv_bfloat16*>(y_slots));
@@ -714,10 +729,12 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
 }
 
 // moe_forward_mxfp4 on the block-scaled tensor cores (mx_tc_supported):
-// chunks of 8 rows per expert for batches of up to 8 tokens, 16 up to 16,
-// else 32.  An expert with more rows than a chunk streams its weights once
-// per chunk.  Stages of 2 K-groups (256 codes, 128 contiguous bytes of every
-// weight row).
+// chunks of 8 rows per expert for batches of up to 8 tokens, else 16.  An
+// expert with more rows than a chunk streams its weights once per chunk (at
+// T = 64 over 16 experts a few do; chunks of 32 rows, which avoid that but
+// fit only two CTAs per SM with a single accumulator, measured 8 % slower).  Several CTAs per SM: each tcgen05 instruction costs its issuing
+// thread a roughly fixed time, so more issuing threads per SM move more
+// bytes (MxTcCfg: CTAs per SM and K-groups per stage by chunk size).
 cudaError_t launch_ffn_decode_mxfp4_tc(const moe_shape& s, const void* x, const int32_t* offsets,
                                        const int32_t* perm, const float* topk_w,
                                        const uint8_t* gu_q, const uint8_t* gu_s,
@@ -725,17 +742,15 @@ cudaError_t launch_ffn_decode_mxfp4_tc(const moe_shape& s, const void* x, const 
                                        uint8_t* xsf, uint8_t* hq, uint8_t* hsf, float* part,
                                        int32_t* ctl, void* y_slots, int32_t* err_flag,
                                        int num_sms, cudaStream_t st) {
-    constexpr int KGS = 2;
     if (!mx_tc_supported(s, gu_q, dn_q) || s.dtype != MOE_BF16 || s.n_shared != 0)
         return cudaErrorInvalidValue;
     if (s.T <= 8)
-        return run_tc<8, KGS>(s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, xq, xsf, hq,
-                              hsf, part, ctl, y_slots, err_flag, num_sms, st);
-    if (s.T <= 16)
-        return run_tc<16, KGS>(s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, xq, xsf, hq,
-                               hsf, part, ctl, y_slots, err_flag, num_sms, st);
-    return run_tc<32, KGS>(s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, xq, xsf, hq, hsf,
-                           part, ctl, y_slots, err_flag, num_sms, st);
+        return run_tc<8, MxTcCfg<8>::KGS, MxTcCfg<8>::CPS>(
+            s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, xq, xsf, hq, hsf, part, ctl,
+            y_slots, err_flag, num_sms, st);
+    return run_tc<16, MxTcCfg<16>::KGS, MxTcCfg<16>::CPS>(
+        s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, xq, xsf, hq, hsf, part, ctl, y_slots,
+        err_flag, num_sms, st);
 }
 
 }  // namespace moe

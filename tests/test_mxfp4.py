@@ -23,7 +23,8 @@ SMALL = [
     MoEConfig("mx_T64_two_chunks", T=64, H=256, I=192, E=4, k=2, zipf_s=1.2),
     MoEConfig("mx_T64_odd_blocks", T=64, H=288, I=160, E=16, k=4, zipf_s=1.0),
     # H and I multiples of 128: the block-scaled tensor-core kernel, chunks of
-    # 8 (T <= 8), 16 (T <= 16) and 32 rows, contraction splits for small batches
+    # 8 (T <= 8) and 16 rows (several per expert at T = 33 and 64),
+    # contraction splits for small batches
     MoEConfig("mx_tc_ragged", T=7, H=512, I=384, E=16, k=3, routed_scale=2.5),
     MoEConfig("mx_tc_k_equals_E", T=8, H=128, I=128, E=4, k=4),
     MoEConfig("mx_tc_T16", T=16, H=384, I=256, E=8, k=2, zipf_s=1.0),
