@@ -157,38 +157,50 @@ __global__ void __launch_bounds__(kBwdThreads) router_backward_kernel(
 
 // Router weight gradient, first pass: part[c][e][h] = sum over the tokens of
 // chunk c of dl[t][e] * x[t][h]; partb[c][e] = sum of dl[t][e].  Block (h
-// chunk of 256, token chunk c); each thread owns one column h and the E
-// experts (in groups of 32 accumulators).
-template <typename XT>
+// chunk of 256, token chunk c); each thread owns one column h and EB experts
+// at a time (EB accumulators, EB >= E where E <= 32).  Chunks are sized so
+// that the grid holds several CTAs per SM (router_wgrad_tokens_per_chunk).
+template <typename XT, int EB>
 __global__ void __launch_bounds__(kBwdThreads) router_wgrad_partial_kernel(
     const XT* __restrict__ x, const float* __restrict__ dl, float* __restrict__ part,
     float* __restrict__ partb, int64_t T, int H, int E, int tokens_per_chunk) {
-    __shared__ float dl_sh[kRouterTokens][33];
+    __shared__ float dl_sh[kRouterTokens][EB + 1];
     const int h = blockIdx.x * kBwdThreads + threadIdx.x;
     const int c = blockIdx.y;
     const int64_t t0 = static_cast<int64_t>(c) * tokens_per_chunk;
     const int64_t t1 = t0 + tokens_per_chunk < T ? t0 + tokens_per_chunk : T;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-        const int ne = E - e0 < 32 ? E - e0 : 32;
-        float acc[32];
+    for (int e0 = 0; e0 < E; e0 += EB) {
+        const int ne = E - e0 < EB ? E - e0 : EB;
+        float acc[EB];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+        for (int j = 0; j < EB; ++j) acc[j] = 0.f;
         float accb = 0.f;
         for (int64_t ts = t0; ts < t1; ts += kRouterTokens) {
             const int nt = t1 - ts < kRouterTokens ? static_cast<int>(t1 - ts) : kRouterTokens;
             __syncthreads();
-            for (int i = threadIdx.x; i < kRouterTokens * 32; i += kBwdThreads) {
-                const int tt = i / 32, j = i % 32;
+            for (int i = threadIdx.x; i < kRouterTokens * EB; i += kBwdThreads) {
+                const int tt = i / EB, j = i % EB;
                 dl_sh[tt][j] = (tt < nt && j < ne) ? dl[(ts + tt) * E + e0 + j] : 0.f;
             }
             __syncthreads();
-            if (threadIdx.x < 32 && blockIdx.x == 0)
+            if (threadIdx.x < EB && blockIdx.x == 0)
                 for (int tt = 0; tt < nt; ++tt) accb += dl_sh[tt][threadIdx.x];
             if (h < H) {
-                for (int tt = 0; tt < nt; ++tt) {
+                int tt = 0;
+                // four token rows' loads in flight at a time
+                for (; tt + 4 <= nt; tt += 4) {
+                    float xv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) xv[u] = ElemIO<XT>::load(x, (ts + tt + u) * H + h);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+#pragma unroll
+                        for (int j = 0; j < EB; ++j) acc[j] = fmaf(dl_sh[tt + u][j], xv[u], acc[j]);
+                }
+                for (; tt < nt; ++tt) {
                     const float xv = ElemIO<XT>::load(x, (ts + tt) * H + h);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[j] = fmaf(dl_sh[tt][j], xv, acc[j]);
+                    for (int j = 0; j < EB; ++j) acc[j] = fmaf(dl_sh[tt][j], xv, acc[j]);
                 }
             }
         }
@@ -277,14 +289,31 @@ cudaError_t launch_expert_backward(const moe_shape&, int64_t, const int32_t*, co
 
 // n-tiles (256 columns of I) of the down-projection dgrad: the per-slot parts
 // of the routing weight's gradient.
-int backward_dw_tiles(const moe_shape& s) { return (s.I + 255) / 256; }
+// routing-weight partials per slot: one per (256-column tile, half of it)
+int backward_dw_tiles(const moe_shape& s) { return 2 * ((s.I + 255) / 256); }
 
 size_t backward_pad_rows(const moe_shape& s) {
     return static_cast<size_t>(s.T * s.k) + static_cast<size_t>(kBwdPad - 1) * s.E;
 }
 
+// Tokens per chunk of the router weight gradient: enough chunks that the
+// (H/256) x chunks grid holds about 600 CTAs, at least 64 tokens a chunk,
+// and the float32 partials within 64 MB.
+int router_wgrad_tokens_per_chunk(const moe_shape& s) {
+    const int64_t hb = (s.H + kBwdThreads - 1) / kBwdThreads;
+    int64_t chunks = (600 + hb - 1) / hb;
+    const int64_t max_by_tokens = (s.T + kRouterTokens - 1) / kRouterTokens;
+    const int64_t max_by_bytes = (64ll << 20) / (static_cast<int64_t>(s.E) * s.H * 4);
+    if (chunks > max_by_tokens) chunks = max_by_tokens;
+    if (chunks > max_by_bytes) chunks = max_by_bytes;
+    if (chunks < 1) chunks = 1;
+    int64_t per = (s.T + chunks - 1) / chunks;
+    per = (per + kRouterTokens - 1) / kRouterTokens * kRouterTokens;
+    return static_cast<int>(per > 0 ? per : kRouterTokens);
+}
+
 int router_wgrad_chunks(const moe_shape& s) {
-    const int64_t per = 1024;
+    const int64_t per = router_wgrad_tokens_per_chunk(s);
     const int64_t n = (s.T + per - 1) / per;
     return static_cast<int>(n > 0 ? n : 1);
 }
@@ -322,13 +351,23 @@ cudaError_t launch_backward(const moe_shape& s, const void* x, const float* w_ro
         aux_coef, backward_dw_tiles(s));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int chunks = router_wgrad_chunks(s);
+    const int tpc = router_wgrad_tokens_per_chunk(s);
     dim3 g1(static_cast<unsigned>((s.H + kBwdThreads - 1) / kBwdThreads), static_cast<unsigned>(chunks));
-    if (s.dtype == MOE_BF16)
-        router_wgrad_partial_kernel<__nv_bfloat16><<<g1, kBwdThreads, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(x), b.dl, b.part, b.partb, s.T, s.H, s.E, 1024);
-    else
-        router_wgrad_partial_kernel<float><<<g1, kBwdThreads, 0, st>>>(
-            static_cast<const float*>(x), b.dl, b.part, b.partb, s.T, s.H, s.E, 1024);
+    if (s.dtype == MOE_BF16) {
+        const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+        if (s.E <= 8)
+            router_wgrad_partial_kernel<__nv_bfloat16, 8><<<g1, kBwdThreads, 0, st>>>(
+                xb, b.dl, b.part, b.partb, s.T, s.H, s.E, tpc);
+        else if (s.E <= 16)
+            router_wgrad_partial_kernel<__nv_bfloat16, 16><<<g1, kBwdThreads, 0, st>>>(
+                xb, b.dl, b.part, b.partb, s.T, s.H, s.E, tpc);
+        else
+            router_wgrad_partial_kernel<__nv_bfloat16, 32><<<g1, kBwdThreads, 0, st>>>(
+                xb, b.dl, b.part, b.partb, s.T, s.H, s.E, tpc);
+    } else {
+        router_wgrad_partial_kernel<float, 32><<<g1, kBwdThreads, 0, st>>>(
+            static_cast<const float*>(x), b.dl, b.part, b.partb, s.T, s.H, s.E, tpc);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t n = static_cast<int64_t>(s.E) * s.H;
     router_wgrad_reduce_kernel<<<static_cast<unsigned>((n + kBwdThreads - 1) / kBwdThreads),

@@ -49,7 +49,8 @@ constexpr int B_BYTES = BN * BK * 2;          // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int BOX_BYTES = 64 * BK * 2;        // one MN-major box: 64 columns x 64 rows
 constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter, each on half the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 }  // namespace bwd
 
@@ -64,6 +65,40 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1) << 46;                    // descriptor version (sm_100)
     d |= static_cast<uint64_t>(2) << 61;                    // swizzle: 128 B
     return d;
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16_bwd(uint32_t taddr, float* v) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// TMA tensor store of a 3D box from shared memory (coordinates innermost
+// first), tracked by the thread's bulk async-group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int32_t c0,
+                                             int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// every committed bulk store of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every committed bulk store of this thread is complete
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 struct BwdParams {
@@ -145,7 +180,12 @@ struct BwdTile {
     int n0;      // first output column
 };
 
-template <int MAXG>
+// Tile order within a group.  kWgrad: n inner (all of an expert's operand
+// rows fit in L2 either way).  dgrad: m inner, so that the CTAs working at
+// the same time share the B panel (a slice of the expert's weight, read once
+// from memory) and re-read only the expert's small A rows from L2; with n
+// inner every m-tile streamed the whole weight again.
+template <int MODE, int MAXG>
 __device__ __forceinline__ BwdTile decode_bwd_tile(const BwdTable<MAXG>& bt, const BwdParams& p,
                                                    int tile) {
     int lo = 0, hi = bt.n_groups - 1;
@@ -158,9 +198,15 @@ __device__ __forceinline__ BwdTile decode_bwd_tile(const BwdTable<MAXG>& bt, con
     c.g = lo;
     c.routed = lo < p.E;
     const int local = tile - bt.tile_start[lo];
-    const int nt = c.routed ? p.n_tiles_routed : p.n_tiles_shared;
-    c.m0 = (local / nt) * bwd::BM;       // n inner: consecutive tiles share the A rows
-    c.n0 = (local % nt) * bwd::BN;
+    if (MODE == kWgrad) {
+        const int nt = c.routed ? p.n_tiles_routed : p.n_tiles_shared;
+        c.m0 = (local / nt) * bwd::BM;
+        c.n0 = (local % nt) * bwd::BN;
+    } else {
+        const int mt = (bt.prows[lo] + bwd::BM - 1) / bwd::BM;
+        c.m0 = (local % mt) * bwd::BM;
+        c.n0 = (local / mt) * bwd::BN;
+    }
     return c;
 }
 
@@ -168,6 +214,7 @@ template <int MODE>
 __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
     const __grid_constant__ CUtensorMap map_a_routed, const __grid_constant__ CUtensorMap map_a_shared,
     const __grid_constant__ CUtensorMap map_b_routed, const __grid_constant__ CUtensorMap map_b_shared,
+    const __grid_constant__ CUtensorMap map_o_routed, const __grid_constant__ CUtensorMap map_o_shared,
     const BwdParams p) {
     using namespace bwd;
     constexpr bool A_MN = MODE == kWgrad;
@@ -176,6 +223,9 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
     __shared__ int32_t offs_sh[kMaxExperts + 1];
     __shared__ int32_t poffs_sh[kMaxExperts + 1];
     __shared__ uint32_t tmem_base_sh;
+    // kWgrad epilogue: per epilogue warp one 32-row x 16-column fp32 block,
+    // 64-byte swizzled, that a TMA tensor store writes out
+    __shared__ __align__(1024) float wg_out[MODE == kWgrad ? EPI_WARPS : 1][32 * 16];
 
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -201,7 +251,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128);
+            mbar_init(&tempty[b], 32 * EPI_WARPS);
         }
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -240,7 +290,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const BwdTile c = decode_bwd_tile(bt, p, tile);
+                const BwdTile c = decode_bwd_tile<MODE>(bt, p, tile);
                 const CUtensorMap* ma = c.routed ? &map_a_routed : &map_a_shared;
                 const CUtensorMap* mb = c.routed ? &map_b_routed : &map_b_shared;
                 const int eidx = c.routed ? c.g : c.g - p.E;
@@ -296,7 +346,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const BwdTile c = decode_bwd_tile(bt, p, tile);
+                const BwdTile c = decode_bwd_tile<MODE>(bt, p, tile);
                 const int nkb = num_kb(c);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, deadline)) { ok = false; break; }
                 tc_fence_after();
@@ -329,10 +379,12 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
         const int r_in_tile = quarter * 32 + lane;
+        const int ch = (warp - 2) >> 2;              // which half of the columns
+        const int c_begin = ch * (BN / 2), c_end = c_begin + BN / 2;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const BwdTile c = decode_bwd_tile(bt, p, tile);
+            const BwdTile c = decode_bwd_tile<MODE>(bt, p, tile);
             if (!mbar_wait(&tfull[acc], acc_phase, deadline)) {
                 raise_error(p.err_flag, MOE_ERR_TIMEOUT);
                 break;
@@ -346,29 +398,37 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
                 const int eidx = c.routed ? c.g : c.g - p.E;
                 const int m = c.m0 + r_in_tile;
                 const bool has_k = num_kb(c) > 0;
-                float* out = static_cast<float*>(c.routed ? p.out_routed : p.out_shared) +
-                             static_cast<int64_t>(eidx) * M * N;
+                // the warp's 32 rows x 16 columns are staged in shared memory
+                // (row = lane, 64-byte swizzle: 16-byte chunk q of row r at
+                // q ^ ((r >> 1) & 3), conflict-free) and written by one TMA
+                // store; rows past M and columns past N fall outside the
+                // tensor map and are not written
+                const CUtensorMap* mo = c.routed ? &map_o_routed : &map_o_shared;
+                float* buf = wg_out[warp - 2];
+                const uint32_t sbuf = smem_u32(buf);
+                (void)M;
 #pragma unroll 1
-                for (int cc = 0; cc < BN; cc += 32) {
-                    float v[32];
+                for (int cc = c_begin; cc < c_end; cc += 16) {
+                    float v[16];
                     if (has_k) {
-                        tmem_ld32(taddr + cc, v);
+                        tmem_ld16_bwd(taddr + cc, v);
                         tmem_ld_wait();
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                        for (int j = 0; j < 16; ++j) v[j] = 0.f;
                     }
-                    const int n = c.n0 + cc;
-                    if (m < M) {
-                        float* dst = out + static_cast<int64_t>(m) * N + n;
+                    // the previous store of this warp has read the buffer
+                    if (lane == 0) bulk_wait_read0();
+                    __syncwarp();
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            if (n + 4 * q + 3 < N)
-                                reinterpret_cast<float4*>(dst)[q] =
-                                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                            else
-                                for (int j = 0; j < 4; ++j)
-                                    if (n + 4 * q + j < N) dst[4 * q + j] = v[4 * q + j];
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<float4*>(buf + lane * 16 + ((q ^ ((lane >> 1) & 3)) * 4)) =
+                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(mo, sbuf, c.n0 + cc, c.m0 + quarter * 32, eidx);
+                        bulk_commit();
                     }
                 }
             } else if (MODE == kDgradDown) {
@@ -387,7 +447,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
                                      orow * 2 * I2;
                 float dwp = 0.f;
 #pragma unroll 1
-                for (int cc = 0; cc < BN; cc += 32) {
+                for (int cc = c_begin; cc < c_end; cc += 32) {
                     float v[32];
                     tmem_ld32(taddr + cc, v);
                     tmem_ld_wait();
@@ -436,7 +496,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
                     }
                 }
                 if (valid && c.routed)
-                    p.dw_raw[static_cast<int64_t>(p.perm[grow]) * p.n_tiles_routed + c.n0 / BN] = dwp;
+                    p.dw_raw[(static_cast<int64_t>(p.perm[grow]) * p.n_tiles_routed + c.n0 / BN) * 2 + ch] = dwp;
             } else {
                 // kDgradGateUp: dx of the slot row (routed: padded row prow0 + m;
                 // shared: s*T + m), bf16
@@ -447,7 +507,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
                                                                           : p.out_shared) +
                                      orow * N;
 #pragma unroll 1
-                for (int cc = 0; cc < BN; cc += 32) {
+                for (int cc = c_begin; cc < c_end; cc += 32) {
                     float v[32];
                     tmem_ld32(taddr + cc, v);
                     tmem_ld_wait();
@@ -470,6 +530,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
         }
     }
 
+    // the TMA stores have finished (they read shared memory that the CTA frees)
+    if (MODE == kWgrad && warp >= 2 && lane == 0) bulk_wait_all();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -477,9 +539,25 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
     }
 }
 
+// Weight gradient [E, M, N] float32 as a 3D tensor (N, M, E) for the
+// epilogue's TMA stores: box 16 columns x 32 rows, 64-byte swizzle.
+static bool make_map_out_f32(CUtensorMap* map, void* base, int E, int64_t M, int64_t N) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc || !base || E <= 0 || M <= 0 || N <= 0 || (N * 4) % 16 != 0) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M),
+                          static_cast<cuuint64_t>(E)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(N * 4), static_cast<cuuint64_t>(M * N * 4)};
+    cuuint32_t box[3] = {16u, 32u, 1u};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int MODE>
 static cudaError_t launch_bwd_mode(const CUtensorMap& a_r, const CUtensorMap& a_s,
                                    const CUtensorMap& b_r, const CUtensorMap& b_s,
+                                   const CUtensorMap& o_r, const CUtensorMap& o_s,
                                    const BwdParams& p, int64_t tiles_bound, int num_sms,
                                    cudaStream_t st) {
     auto kern = grouped_gemm_bwd<MODE>;
@@ -488,7 +566,7 @@ static cudaError_t launch_bwd_mode(const CUtensorMap& a_r, const CUtensorMap& a_
     if (e != cudaSuccess) return e;
     const int grid = static_cast<int>(tiles_bound < num_sms ? (tiles_bound > 0 ? tiles_bound : 1)
                                                             : num_sms);
-    kern<<<grid, bwd::THREADS, bwd::SMEM_BYTES, st>>>(a_r, a_s, b_r, b_s, p);
+    kern<<<grid, bwd::THREADS, bwd::SMEM_BYTES, st>>>(a_r, a_s, b_r, b_s, o_r, o_s, p);
     return cudaGetLastError();
 }
 
@@ -553,7 +631,7 @@ cudaError_t launch_expert_backward(const moe_shape& s, int64_t P, const int32_t*
         p.out_routed = dgu;
         p.out_shared = dgu_sh;
         cudaError_t e = launch_bwd_mode<kDgradDown>(
-            ar, as, br, bs, p, mt_dgrad * (p.n_tiles_routed > p.n_tiles_shared ? p.n_tiles_routed
+            ar, as, br, bs, ar, ar, p, mt_dgrad * (p.n_tiles_routed > p.n_tiles_shared ? p.n_tiles_routed
                                                                                 : p.n_tiles_shared),
             num_sms, st);
         if (e != cudaSuccess) return e;
@@ -585,7 +663,11 @@ cudaError_t launch_expert_backward(const moe_shape& s, int64_t P, const int32_t*
         p.b_sh_stride = s.T;        // h_sh rows s*T + t
         const int64_t tiles = static_cast<int64_t>(E) * p.m_tiles_routed * p.n_tiles_routed +
                               static_cast<int64_t>(S) * p.m_tiles_shared * p.n_tiles_shared;
-        cudaError_t e = launch_bwd_mode<kWgrad>(ar, as, br, bs, p, tiles, num_sms, st);
+        CUtensorMap orr, os;
+        if (!make_map_out_f32(&orr, d_down, E, H, I) ||
+            !make_map_out_f32(&os, S > 0 ? d_sh_down : d_down, S > 0 ? S : E, H, S > 0 ? Is : I))
+            return cudaErrorInvalidValue;
+        cudaError_t e = launch_bwd_mode<kWgrad>(ar, as, br, bs, orr, os, p, tiles, num_sms, st);
         if (e != cudaSuccess) return e;
     }
     // ---- 3. dgrad through gate_up: dX (into dO's buffer, which is dead by now)
@@ -611,7 +693,7 @@ cudaError_t launch_expert_backward(const moe_shape& s, int64_t P, const int32_t*
         p.b_rows_shared = 2 * Is;
         p.out_routed = dX;
         p.out_shared = dX_sh;
-        cudaError_t e = launch_bwd_mode<kDgradGateUp>(ar, as, br, bs, p,
+        cudaError_t e = launch_bwd_mode<kDgradGateUp>(ar, as, br, bs, ar, ar, p,
                                                       mt_dgrad * p.n_tiles_routed, num_sms, st);
         if (e != cudaSuccess) return e;
     }
@@ -642,7 +724,12 @@ cudaError_t launch_expert_backward(const moe_shape& s, int64_t P, const int32_t*
         p.b_sh_stride = 0;          // x rows
         const int64_t tiles = static_cast<int64_t>(E) * p.m_tiles_routed * p.n_tiles_routed +
                               static_cast<int64_t>(S) * p.m_tiles_shared * p.n_tiles_shared;
-        return launch_bwd_mode<kWgrad>(ar, as, br, bs, p, tiles, num_sms, st);
+        CUtensorMap orr, os;
+        if (!make_map_out_f32(&orr, d_gate_up, E, 2 * I, H) ||
+            !make_map_out_f32(&os, S > 0 ? d_sh_gate_up : d_gate_up, S > 0 ? S : E,
+                              S > 0 ? 2 * Is : 2 * I, H))
+            return cudaErrorInvalidValue;
+        return launch_bwd_mode<kWgrad>(ar, as, br, bs, orr, os, p, tiles, num_sms, st);
     }
 }
 
