@@ -101,6 +101,19 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// 16-byte load, zero when !ok; volatile so that it is issued where written
+// (ahead of the math that consumes it).
+__device__ __forceinline__ uint4 ldg16_pred(const __nv_bfloat16* ptr, bool ok) {
+    uint4 v;
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+        "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+        "@q ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(ptr), "r"(static_cast<int>(ok)));
+    return v;
+}
+
 struct BwdParams {
     const int32_t* offsets;    // [E+1] sorted rows of each routed expert
     const int32_t* poffsets;   // [E+1] the same, each expert padded to a multiple of 128
@@ -446,10 +459,24 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
                                                                           : p.out_shared) +
                                      orow * 2 * I2;
                 float dwp = 0.f;
+                // g and u of the next 32 columns are requested before this
+                // chunk's tensor-memory load and math, so their latency hides
+                uint4 gcur[4], ucur[4], gnxt[4], unxt[4];
+                auto load_gu = [&](int cc, uint4 (&g4)[4], uint4 (&u4)[4]) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int nq = c.n0 + cc + 8 * q;
+                        const bool in = valid && nq < N;
+                        g4[q] = ldg16_pred(gu + nq, in);
+                        u4[q] = ldg16_pred(gu + I2 + nq, in);
+                    }
+                };
+                load_gu(c_begin, gcur, ucur);
 #pragma unroll 1
                 for (int cc = c_begin; cc < c_end; cc += 32) {
                     float v[32];
                     tmem_ld32(taddr + cc, v);
+                    if (cc + 32 < c_end) load_gu(cc + 32, gnxt, unxt);
                     tmem_ld_wait();
                     const int n = c.n0 + cc;
                     if (valid) {
@@ -457,8 +484,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
                         for (int q = 0; q < 4; ++q) {
                             const int nq = n + 8 * q;
                             if (nq >= N) break;
-                            const uint4 gv = *reinterpret_cast<const uint4*>(gu + nq);
-                            const uint4 uv = *reinterpret_cast<const uint4*>(gu + I2 + nq);
+                            const uint4 gv = gcur[q];
+                            const uint4 uv = ucur[q];
                             const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
                             const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
                             uint32_t og[4], ou[4];
@@ -493,6 +520,11 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
                             *reinterpret_cast<uint4*>(dgu + nq) = make_uint4(0, 0, 0, 0);
                             *reinterpret_cast<uint4*>(dgu + I2 + nq) = make_uint4(0, 0, 0, 0);
                         }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        gcur[q] = gnxt[q];
+                        ucur[q] = unxt[q];
                     }
                 }
                 if (valid && c.routed)
