@@ -111,10 +111,7 @@ __global__ void __launch_bounds__(256) combine_bf16_pipelined_kernel(
 
 cudaError_t launch_combine(const moe_shape& s, const void* y_slots, const int32_t* inv, void* y,
                            cudaStream_t st) {
-#ifndef MOE_COMBINE_PIPELINED
-#define MOE_COMBINE_PIPELINED 1
-#endif
-    if (MOE_COMBINE_PIPELINED && s.dtype == MOE_BF16) {
+    if (s.dtype == MOE_BF16) {
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) == cudaSuccess)
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

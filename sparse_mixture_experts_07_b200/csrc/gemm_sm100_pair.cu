@@ -121,13 +121,11 @@ __global__ void __launch_bounds__(pair::THREADS, 1) grouped_gemm_pair(
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
-#ifndef MOE_PAIR_L2_HINTS
-#define MOE_PAIR_L2_HINTS 1
-#endif
             // L2 priorities: activation rows are reused by every n-tile of their
-            // group, weight panels only by the few m-tiles of one band
-            const uint64_t pol_a = MOE_PAIR_L2_HINTS ? l2_policy_evict_last() : l2_policy_evict_normal();
-            const uint64_t pol_b = MOE_PAIR_L2_HINTS >= 2 ? l2_policy_evict_first() : l2_policy_evict_normal();
+            // group (evict-last); weight panels keep the normal policy
+            // (evict-first on them measured 8-15 % slower)
+            const uint64_t pol_a = l2_policy_evict_last();
+            const uint64_t pol_b = l2_policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;

@@ -392,17 +392,13 @@ moe_status forward_range(const moe_shape& s, int e_begin, int e_end, bool with_s
     // CTA pairs (256-row tiles) when the experts average at least 256 rows;
     // one CTA per tile otherwise (less padding on small groups).  The average
     // is over all E experts, a range's share of the rows being proportional.
-#ifndef MOE_PAIR_MIN_ROWS
-#define MOE_PAIR_MIN_ROWS 256
-#endif
-#ifndef MOE_PAIR_GROUP_M
-#define MOE_PAIR_GROUP_M 16
-#endif
-    if (s.T * s.k >= static_cast<int64_t>(MOE_PAIR_MIN_ROWS) * s.E)
+    constexpr int kPairMinRows = 256;   // average rows per expert for CTA pairs
+    constexpr int kPairGroupM = 16;     // m-tiles per rasterisation band
+    if (s.T * s.k >= static_cast<int64_t>(kPairMinRows) * s.E)
         return cuda_status(moe::launch_ffn_sm100_pair(sl, x, x_perm, offs, perm, topk_w, gate_up,
                                                       down, sh_gate_up, sh_down, h_routed,
                                                       h_shared, y_slots, err_flag, sms,
-                                                      MOE_PAIR_GROUP_M, cs, gu_routed, gu_shared));
+                                                      kPairGroupM, cs, gu_routed, gu_shared));
     return cuda_status(moe::launch_ffn_sm100(sl, x, x_perm, offs, perm, topk_w, gate_up, down,
                                              sh_gate_up, sh_down, h_routed, h_shared, y_slots,
                                              err_flag, sms, 8, cs, gu_routed, gu_shared));

@@ -29,6 +29,9 @@ SMALL = [
     # > 256 tokens: tensor-core router (E <= 64) or CUDA-core tiled router
     MoEConfig("f32_many_tokens", T=600, H=72, I=64, E=8, k=2, dtype="f32"),
     MoEConfig("bf16_E128", T=300, H=128, I=64, E=128, k=4),
+    # decode-batch router cluster with the router slice read from memory (E x H/8
+    # floats do not fit in shared memory), 256 experts
+    MoEConfig("bf16_route_cluster_E256", T=20, H=2048, I=64, E=256, k=8),
     MoEConfig("bf16_router_tc_E40", T=520, H=200, I=64, E=40, k=3, zipf_s=1.0),
     # decode batches (T <= 8) take the weight-streaming path; ragged H, I, Is
     MoEConfig("bf16_decode_shared", T=7, H=712, I=328, E=16, k=3, n_shared=2, I_shared=200,
