@@ -323,6 +323,14 @@ class Workload:
                                       d["down"], d["sh_gate_up"], d["sh_down"])
         self.x = d["x"]
 
+    def touched_bytes(self) -> float:
+        """Bytes one step must read at least: the active experts' weights for a
+        decode batch (from the plan of the last step), all weights otherwise."""
+        if self.cfg.T * self.cfg.k <= 256:
+            counts = self.layer.buf["counts"].cpu().numpy()
+            return bytes_decode(self.cfg, counts, mxfp4=self.mx is not None)
+        return float(self.weight_bytes())
+
     def weight_bytes(self) -> int:
         if self.mx is not None:
             return sum(v.numel() for v in self.mx.values())
@@ -331,6 +339,18 @@ class Workload:
         if self.inp["sh_gate_up"] is not None:
             n += self.inp["sh_gate_up"].numel() + self.inp["sh_down"].numel()
         return n * eb
+
+    def forward(self, stream=None):
+        """The moe_forward region alone, on the plan the last step left in the buffers."""
+        moe, s, L = self.moe, self.shape, self.layer
+        b = L.buf
+        if self.mx is not None:
+            moe.forward_mxfp4(s, self.x, b["offsets"], b["perm"], b["topk_w"], self.mx,
+                              L.workspace, L.err_flag, y_slots=b["y_slots"], stream=stream)
+        else:
+            moe.forward(s, self.x, b["offsets"], b["perm"], b["topk_w"], L.gate_up, L.down,
+                        L.sh_gate_up, L.sh_down, L.workspace, L.err_flag, y_slots=b["y_slots"],
+                        stream=stream)
 
     def step(self, stream, fwd_start=None, fwd_end=None):
         """route -> permute -> forward -> combine, with events around the forward."""
@@ -341,12 +361,7 @@ class Workload:
         moe.permute(s, idx, L.workspace, L.err_flag, out=b, stream=stream)
         if fwd_start is not None:
             fwd_start.record(stream)
-        if self.mx is not None:
-            moe.forward_mxfp4(s, self.x, b["offsets"], b["perm"], w, self.mx, L.workspace,
-                              L.err_flag, y_slots=b["y_slots"], stream=stream)
-        else:
-            moe.forward(s, self.x, b["offsets"], b["perm"], w, L.gate_up, L.down, L.sh_gate_up,
-                        L.sh_down, L.workspace, L.err_flag, y_slots=b["y_slots"], stream=stream)
+        self.forward(stream)
         if fwd_end is not None:
             fwd_end.record(stream)
         moe.combine(s, b["y_slots"], b["inv"], y=b["y"], stream=stream)
@@ -361,6 +376,39 @@ EXTRA_WORKLOADS = [
 ]
 
 
+def measure_graph(w, stream, steps, flush) -> dict:
+    """Decode batches replayed from CUDA graphs: the whole step (MoEGraph, the
+    layer's public capture) and the moe_forward region alone, each replay timed
+    with CUDA events on `stream`, the L2 flushed first when `flush` is given.
+    Without the host's per-launch cost the forward region shows the kernels'
+    own device time."""
+    step_graph = w.layer.capture(w.x)
+    side = torch.cuda.Stream(device=w.x.device)
+    side.wait_stream(stream)
+    fwd_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(fwd_graph, stream=side):
+        w.forward()
+    stream.wait_stream(side)
+    times = {}
+    for key, g in (("ms_per_step", step_graph.graph), ("forward_ms", fwd_graph)):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for _ in range(3):
+            g.replay()
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            ev[i][0].record(stream)
+            g.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        times[key] = statistics.median(a.elapsed_time(b) for a, b in ev)
+    assert w.layer.device_error() == 0, "device error flag set (graph replay)"
+    del step_graph, fwd_graph
+    return {"graph": {"ms_per_step": times["ms_per_step"],
+                      "tokens_per_s": w.cfg.T / (times["ms_per_step"] / 1000.0),
+                      "forward_ms": times["forward_ms"]}}
+
+
 def measure_extra(name, weights, dev, steps, peaks, flush) -> dict:
     """Device time of `steps` steps of one workload, each step timed on its own
     with the L2 flushed in between when the step's weights would fit in L2."""
@@ -371,7 +419,8 @@ def measure_extra(name, weights, dev, steps, peaks, flush) -> dict:
         w.step(stream)
     torch.cuda.synchronize()
     assert w.layer.device_error() == 0, f"device error flag set ({name})"
-    need_flush = w.weight_bytes() < 4 * L2_BYTES
+    touched = w.touched_bytes()
+    need_flush = touched < 4 * L2_BYTES
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for i in range(steps):
         if need_flush:
@@ -386,13 +435,18 @@ def measure_extra(name, weights, dev, steps, peaks, flush) -> dict:
     fwd_ms = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
     counts = w.layer.buf["counts"].cpu().numpy()
     roof = roofline_of(cfg, counts, fwd_ms, 0.0, w.mx is not None, peaks)
+    keys = ("bound", "achieved", "peak", "unit", "frac", "peak_kind")
     out = {"workload": name, "weights": weights, "T": cfg.T, "steps": steps,
            "ms_per_step": step_ms, "tokens_per_s": cfg.T / (step_ms / 1000.0),
-           "forward_ms": fwd_ms, "roofline": {k: roof[k] for k in (
-               "bound", "achieved", "peak", "unit", "frac", "peak_kind")},
-           "l2": "L2 flushed before every step (256 MB write)" if need_flush
-                 else f"weights {w.weight_bytes() / 1e9:.2f} GB > L2, streamed every step",
+           "forward_ms": fwd_ms, "roofline": {k: roof[k] for k in keys},
+           "l2": f"L2 flushed before every step (256 MB write; {touched / 1e9:.3f} GB "
+                 "touched per step)" if need_flush
+                 else f"weights touched per step {touched / 1e9:.2f} GB > 4x L2, streamed",
            "active_experts": int((counts > 0).sum())}
+    if cfg.T * cfg.k <= 256:
+        out.update(measure_graph(w, stream, steps, flush if need_flush else None))
+        groof = roofline_of(cfg, counts, out["graph"]["forward_ms"], 0.0, w.mx is not None, peaks)
+        out["graph"]["roofline"] = {k: groof[k] for k in keys}
     del w
     torch.cuda.empty_cache()
     return out
@@ -472,11 +526,17 @@ def run_cuda(args, cfg, rank, local, world):
     torch.cuda.synchronize()
     assert layer.device_error() == 0, "device error flag set"
 
-    # ---- device-timed region: K steps, inputs resident in HBM
+    # ---- device-timed region: K steps, inputs resident in HBM.  When the bytes
+    # a step touches would fit in L2 (a small decode batch on MXFP4 weights),
+    # the L2 is flushed before every step and the steps are timed one by one.
     n_ev = args.steps
     fwd_start = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     fwd_end = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     b = layer.buf
+    touched = wl.touched_bytes()
+    flush_l2 = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) \
+        if touched < 4 * L2_BYTES else None
+    step_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_ev)]
     s0 = torch.cuda.Event(enable_timing=True)
     s1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -484,11 +544,18 @@ def run_cuda(args, cfg, rank, local, world):
     with ClockSampler(local) as clk:
         s0.record(stream)
         for i in range(args.steps):
+            if flush_l2 is not None:
+                flush_l2.zero_()
+                step_ev[i][0].record(stream)
             wl.step(stream, fwd_start[i], fwd_end[i])
+            if flush_l2 is not None:
+                step_ev[i][1].record(stream)
         s1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    ms_local = s0.elapsed_time(s1)
+    ms_local = s0.elapsed_time(s1) if flush_l2 is None else \
+        sum(e0.elapsed_time(e1) for e0, e1 in step_ev)
+    del flush_l2
     fwd_ms = statistics.mean(fwd_start[i].elapsed_time(fwd_end[i]) for i in range(n_ev))
     ms_total = max_over_ranks(ms_local, world)
     tokens = cfg.T * args.steps * world
@@ -567,8 +634,11 @@ def run_cuda(args, cfg, rank, local, world):
                    "k": cfg.k, "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
                    "routed_scale": cfg.routed_scale, "weights": weights_label(args, cfg),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (expert weights "
-                         f"{wl.weight_bytes() / 1e9:.2f} GB streamed every step)"},
+                   "l2": "L2 flushed before every step (its touched bytes, "
+                         f"{touched / 1e9:.3f} GB, would fit in 4x L2); steps timed one by one"
+                         if touched < 4 * L2_BYTES else
+                         "inputs larger than L2 (expert weights touched per step "
+                         f"{touched / 1e9:.2f} GB, streamed every step)"},
         "tflops": 2.0 * cfg.T * (cfg.H * cfg.E + 3 * cfg.k * cfg.H * cfg.I +
                                  3 * cfg.n_shared * cfg.I_shared * cfg.H) * args.steps * world /
                   (ms_total / 1000.0) / 1e12,

@@ -226,7 +226,7 @@ def forward(shape: Shape, x, offsets, perm, topk_w, gate_up, down, sh_gate_up, s
 
 def forward_mxfp4(shape: Shape, x, offsets, perm, topk_w, mxfp4: dict, workspace, err_flag,
                   y_slots=None, stream=None):
-    """moe_forward with MXFP4 routed-expert weights (decode batches, T <= 8):
+    """moe_forward with MXFP4 routed-expert weights (decode batches, T <= 64):
     `mxfp4` holds gate_up_q, gate_up_s, down_q, down_s (uint8 device tensors)."""
     lib = load_library()
     if y_slots is None:
@@ -420,3 +420,44 @@ class MoELayer:
     def device_error(self) -> int:
         """Device-detected error bits (synchronises)."""
         return int(self.err_flag.item())
+
+    def capture(self, x, pool=None) -> "MoEGraph":
+        """This layer's step on the static input `x` as a CUDA graph (MoEGraph)."""
+        return MoEGraph(self, x, pool=pool)
+
+
+class MoEGraph:
+    """One MoELayer step (route, permute, forward, combine) captured once as a
+    CUDA graph.
+
+    Every launch of the step reads its shapes from the host and its routing
+    from device buffers, so a graph replays the step exactly: write the next
+    tokens into the static `x` (same shape, same storage) and call replay(),
+    which leaves y [T, H] in `y` (the layer's output buffer).  Worth it for
+    decode batches, where the step's launches cost about as much as streaming
+    the active experts' weights.  The layer's buffers and workspace are shared
+    with its eager calls; do not run both at once on different streams.
+    """
+
+    def __init__(self, layer: MoELayer, x, pool=None):
+        if x.shape != (layer.shape.T, layer.shape.H):
+            raise ValueError(f"x must be [{layer.shape.T}, {layer.shape.H}], got {tuple(x.shape)}")
+        self.layer, self.x, self.y = layer, x, layer.buf["y"]
+        dev = x.device
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            layer(x)  # first launches set kernel attributes outside the capture
+        torch.cuda.current_stream(dev).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, pool=pool, stream=side):
+            layer(x)
+
+    def replay(self, stream=None):
+        """Run the captured step on `stream` (default: the current stream); returns y."""
+        if stream is None:
+            self.graph.replay()
+        else:
+            with torch.cuda.stream(stream):
+                self.graph.replay()
+        return self.y
