@@ -73,6 +73,8 @@ __global__ void __launch_bounds__(256) combine_bf16_pipelined_kernel(
     const int64_t routed_rows = n_tokens * k;
     const int nrows = k + S;
     int64_t t = blockIdx.x;
+    pdl_launch_dependents();     // launched as a programmatic dependent
+    pdl_wait();
     // the threads < k fetch one slot index each for the next token
     int32_t next_idx = (t < n_tokens && static_cast<int>(threadIdx.x) < k)
                            ? inv[t * k + threadIdx.x] : 0;
@@ -117,10 +119,9 @@ cudaError_t launch_combine(const moe_shape& s, const void* y_slots, const int32_
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int64_t cap = static_cast<int64_t>(sms) * 8;    // 8 CTAs of 256 threads per SM
         const unsigned grid = static_cast<unsigned>(s.T < cap ? s.T : cap);
-        combine_bf16_pipelined_kernel<<<grid, 256, 0, st>>>(
-            static_cast<const uint4*>(y_slots), inv, static_cast<uint4*>(y), s.T, s.H / 8, s.k,
-            s.n_shared);
-        return cudaGetLastError();
+        return launch_pdl(combine_bf16_pipelined_kernel, dim3(grid), dim3(256), 0, st,
+                          static_cast<const uint4*>(y_slots), inv, static_cast<uint4*>(y), s.T,
+                          s.H / 8, s.k, s.n_shared);
     }
     const unsigned grid = static_cast<unsigned>(s.T < 1048576 ? s.T : 1048576);
     if (s.dtype == MOE_BF16) {

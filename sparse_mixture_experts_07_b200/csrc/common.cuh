@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -92,6 +94,36 @@ using GroupTable = GroupTableT<kMaxGroups>;
 // PTX wrappers (sm_100a).
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Programmatic dependent launch (the decode chain: router, plan, decode
+// expert kernels, combine).  A kernel launched by launch_pdl may begin while
+// the kernel before it in the stream is still running.  It calls
+// pdl_launch_dependents() on entry, so that the kernel after it may be
+// scheduled early in turn, and pdl_wait() before it first touches memory
+// that an earlier kernel writes or reads: pdl_wait returns once the previous
+// kernel has completed and its writes are visible, and since that kernel
+// waited the same way, every earlier one has too.  A kernel launched the
+// ordinary way finds both instructions without effect.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 __device__ __forceinline__ uint64_t global_ns() {

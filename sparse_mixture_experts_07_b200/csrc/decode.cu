@@ -44,9 +44,12 @@ struct DecodeParams {
 };
 
 // One CTA per work unit (grid-stride); its 4 warps split the contraction.
+// Both kernels wait for the previous kernel (pdl_wait) and let the next one
+// launch as they drain; decode_down runs as a programmatic dependent.
 __global__ void __launch_bounds__(dec::THREADS, 2) decode_gate_up_kernel(const DecodeParams p) {
     __shared__ ActiveGroups act;
     __shared__ float red[dec::WARPS * 8 * 32];
+    pdl_wait();
     stage_offsets(act.offs, p.offsets, p.E);
     __syncthreads();
     if (threadIdx.x == 0) build_active(act, p.E, p.S, p.T, p.I, p.Is);
@@ -109,11 +112,17 @@ __global__ void __launch_bounds__(dec::THREADS, 2) decode_gate_up_kernel(const D
             }
         }
     }
+    // the next kernel is let in only as this one drains: its CTAs would
+    // otherwise sit on the SMs through this kernel's second round of CTAs
+    pdl_launch_dependents();
 }
 
-__global__ void __launch_bounds__(dec::THREADS, 2) decode_down_kernel(const DecodeParams p) {
+// Four CTAs per SM (at most 128 registers): with one token the kernel has
+// 2 x H/16 units, which three CTAs per SM would run in two rounds.
+__global__ void __launch_bounds__(dec::THREADS, 4) decode_down_kernel(const DecodeParams p) {
     __shared__ ActiveGroups act;
     __shared__ float red[dec::WARPS * 4 * 32];
+    pdl_wait();
     stage_offsets(act.offs, p.offsets, p.E);
     __syncthreads();
     if (threadIdx.x == 0) build_active(act, p.E, p.S, p.T, p.H, p.H);
@@ -170,6 +179,7 @@ __global__ void __launch_bounds__(dec::THREADS, 2) decode_down_kernel(const Deco
             }
         }
     }
+    pdl_launch_dependents();   // as in decode_gate_up
 }
 
 // Decode path of moe_forward: T <= 8 so every group has at most 8 rows.
@@ -199,12 +209,17 @@ cudaError_t launch_ffn_decode(const moe_shape& s, const void* x, const int32_t* 
     p.S = s.n_shared;
     p.Is = s.n_shared > 0 ? s.I_shared : s.I;
     p.routed_scale = s.routed_scale;
-    const int grid = num_sms * 4;   // 4 CTAs (16 warps) per SM stream weights
+    // 4 CTAs per SM: all resident for decode_down; decode_gate_up (about
+    // 216 registers a thread) holds 2 per SM and takes the rest as they finish.
+    // decode_gate_up is launched the ordinary way: as a programmatic dependent
+    // its CTAs became resident while the router was still running, and its
+    // own run at T = 8 (PhiMoE shape) took 15 % longer (measured; cause not
+    // identified).  decode_down and the combine follow as dependents.
+    const int grid = num_sms * 4;
     decode_gate_up_kernel<<<grid, dec::THREADS, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_down_kernel<<<grid, dec::THREADS, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(decode_down_kernel, dim3(grid), dim3(dec::THREADS), 0, st, p);
 }
 
 }  // namespace moe

@@ -269,17 +269,14 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
     uint64_t* drain = tempty + 2;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint64_t deadline = global_ns() + p.timeout_ns;
     const int nblk = p.K / 32;
     const int n_kg = p.K / KG;                  // K-groups of a whole contraction
 
-    stage_offsets(act.offs, p.offsets, p.E);
-    __syncthreads();
+    // launched as a programmatic dependent: barriers, descriptor prefetch and
+    // tensor memory are set up while the previous kernel finishes; global
+    // memory is touched only after pdl_wait
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
-        build_mx_units(act, p.E, CH, p.mtiles);
-        const int s = mx_tc_splits(act.total_units, gridDim.x, n_kg, KGS, p.S, p.n_out);
-        splits_sh = s;
-        if (blockIdx.x == 0) p.ctl[0] = s;
         for (int i = 0; i < G::STAGES; ++i) {
             mbar_init(&full[i], 1 + 32);    // expect_tx arrival + one cp.async arrival per lane
             mbar_init(&empty[i], 1);        // tcgen05.commit
@@ -296,6 +293,16 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, G::TMEM_COLS);
         tmem_relinquish();
+    }
+    pdl_wait();
+    const uint64_t deadline = global_ns() + p.timeout_ns;
+    stage_offsets(act.offs, p.offsets, p.E);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        build_mx_units(act, p.E, CH, p.mtiles);
+        const int s = mx_tc_splits(act.total_units, gridDim.x, n_kg, KGS, p.S, p.n_out);
+        splits_sh = s;
+        if (blockIdx.x == 0) p.ctl[0] = s;
     }
     tc_fence_before();
     __syncthreads();
@@ -549,6 +556,8 @@ __device__ __forceinline__ void store_e4m3_pair(float v, int64_t r, int blk, int
 __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_prep_x_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int k, int K, int SP,
     uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int r = blockIdx.y;
     const int blk = blockIdx.x * (mxtc::PREP_THREADS / 32) + (threadIdx.x >> 5);
     if (blk >= K / 32) return;
@@ -562,6 +571,8 @@ __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_prep_x_kernel(
 __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_swiglu_kernel(
     const float* __restrict__ part, const int32_t* __restrict__ ctl, int S, int I, int SP,
     uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int r = blockIdx.y;
     const int blk = blockIdx.x * (mxtc::PREP_THREADS / 32) + (threadIdx.x >> 5);
     if (blk >= I / 32) return;
@@ -582,6 +593,8 @@ __global__ void __launch_bounds__(256) mx_tc_down_out_kernel(
     const float* __restrict__ part, const int32_t* __restrict__ ctl, const int32_t* __restrict__ perm,
     const float* __restrict__ topk_w, float routed_scale, int S, int H,
     __nv_bfloat16* __restrict__ y_slots) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int r = blockIdx.y;
     const int n = blockIdx.x * 256 + threadIdx.x;
     if (n >= H) return;
@@ -663,8 +676,7 @@ static cudaError_t launch_tc(const CUtensorMap& mw, const CUtensorMap& ma, const
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          G::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<CPS * num_sms, mxtc::THREADS, G::SMEM_BYTES, st>>>(mw, ma, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(CPS * num_sms), dim3(mxtc::THREADS), G::SMEM_BYTES, st, mw, ma, p);
 }
 
 template <int CH, int KGS, int CPS>
@@ -686,9 +698,9 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
         return cudaErrorInvalidValue;
 
     constexpr int WPB = mxtc::PREP_THREADS / 32;
-    mx_tc_prep_x_kernel<<<dim3((s.H / 32 + WPB - 1) / WPB, S), mxtc::PREP_THREADS, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), perm, s.k, s.H, SP, xq, xsf);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(mx_tc_prep_x_kernel, dim3((s.H / 32 + WPB - 1) / WPB, S),
+                               dim3(mxtc::PREP_THREADS), 0, st,
+                               static_cast<const __nv_bfloat16*>(x), perm, s.k, s.H, SP, xq, xsf);
     if (e != cudaSuccess) return e;
 
     MxTcParams p{};
@@ -710,9 +722,8 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
     p.mtiles = s.I / mxtc::HALF_ROWS;
     e = launch_tc<0, CH, KGS, CPS>(map_gu, map_x, p, num_sms, st);
     if (e != cudaSuccess) return e;
-    mx_tc_swiglu_kernel<<<dim3((s.I / 32 + WPB - 1) / WPB, S), mxtc::PREP_THREADS, 0, st>>>(
-        part, ctl, S, s.I, SP, hq, hsf);
-    e = cudaGetLastError();
+    e = launch_pdl(mx_tc_swiglu_kernel, dim3((s.I / 32 + WPB - 1) / WPB, S),
+                   dim3(mxtc::PREP_THREADS), 0, st, part, ctl, S, s.I, SP, hq, hsf);
     if (e != cudaSuccess) return e;
     // GEMM 2: down, K = I, 128 rows per tile
     p.w_scales = dn_s;
@@ -723,9 +734,9 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
     p.mtiles = s.H / 128;
     e = launch_tc<1, CH, KGS, CPS>(map_dn, map_h, p, num_sms, st);
     if (e != cudaSuccess) return e;
-    mx_tc_down_out_kernel<<<dim3((s.H + 255) / 256, S), 256, 0, st>>>(
-        part, ctl, perm, topk_w, s.routed_scale, S, s.H, static_cast<__nv_bfloat16*>(y_slots));
-    return cudaGetLastError();
+    return launch_pdl(mx_tc_down_out_kernel, dim3((s.H + 255) / 256, S), dim3(256), 0, st, part,
+                      ctl, perm, topk_w, s.routed_scale, S, s.H,
+                      static_cast<__nv_bfloat16*>(y_slots));
 }
 
 // moe_forward_mxfp4 on the block-scaled tensor cores (mx_tc_supported):

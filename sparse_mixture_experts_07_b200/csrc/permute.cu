@@ -170,9 +170,13 @@ __global__ void __launch_bounds__(kPcThreads, 1) permute_cluster_kernel(
     const int64_t lo = rank * chunk;
     const int64_t hi = lo + chunk < n ? lo + chunk : n;
 
+    // launched as a programmatic dependent: shared memory is cleared while
+    // the router finishes, its indices read after pdl_wait
+    pdl_launch_dependents();
     for (int e = tid; e < E; e += kPcThreads) hist[e] = 0;
     for (int i = tid; i < kPcWarps * kMaxExperts; i += kPcThreads)
         (&wcnt[0][0])[i] = -1;                                  // stamp -1: no round
+    pdl_wait();
     __syncthreads();
     // this thread's slots, one per round, kept in registers
     int ev[ROUNDS];
@@ -272,13 +276,15 @@ static cudaError_t launch_permute_cluster_t(const moe_shape& s, int csize, int64
     cfg.blockDim = dim3(kPcThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, permute_cluster_kernel<ROUNDS>, idx, s.T * s.k, s.E, chunk,
                               counts, offsets, perm, inv, err_flag);
 }

@@ -237,10 +237,13 @@ __global__ void __launch_bounds__(256) route_small_kernel(
 
 // Decode batches (at most kRouteClusterTokens tokens per cluster): a cluster
 // of kRouteCluster CTAs per block of tokens, CTA r owning hidden columns
-// [r HS, (r+1) HS).  Each CTA stages its slice of the tokens' rows in shared
-// memory and computes the partial logits of every (token, expert) over its
-// slice (warp w: experts w, w+8, ...; 16-byte loads of the router weights,
-// lane partials summed by a butterfly).  After a cluster barrier, CTA 0 adds
+// [r HS, (r+1) HS).  Each CTA stages its slice of the tokens' rows and of the
+// router weights in shared memory (16-byte cp.async, all in flight at once)
+// and computes the partial logits of every (token, expert) over its slice
+// (warp w: experts w, w+8, ...; one pass over a weight slice for all the
+// block's tokens, lane partials summed by a butterfly).  TBM is the block's
+// token capacity: 1 for a single token (no per-token guards), else
+// kRouteClusterTokens.  After a cluster barrier, CTA 0 adds
 // the kRouteCluster partials of each logit in rank order through distributed
 // shared memory, adds the bias and selects as above; a second barrier keeps
 // the other CTAs' shared memory alive until it has read it.  The router
@@ -261,15 +264,18 @@ __device__ __forceinline__ void cp_async16_route(void* dst, const void* src) {
                  : "memory");
 }
 
-template <typename T>
+template <typename T, int TBM>
 __global__ void __launch_bounds__(256) route_cluster_kernel(
     const T* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
     float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    int64_t n_tokens, int H, int E, int k, int HS, int stage_w) {
+    int64_t n_tokens, int H, int E, int k, int HS, int stage_w, int vec_x) {
     extern __shared__ float4 smem_f4[];
     float* part = reinterpret_cast<float*>(smem_f4);              // [TB][E] partial logits
     float* xs = part + ((kRouteClusterTokens * E + 3) & ~3);      // [TB][HS]
     float* ws = xs + kRouteClusterTokens * HS;                    // [E][HS] if stage_w
+    // bf16 token rows as loaded, [TB][HS], when vec_x (float rows load into xs)
+    T* xb = sizeof(T) == 4 ? reinterpret_cast<T*>(xs)
+                           : reinterpret_cast<T*>(stage_w ? ws + E * HS : ws);
     const uint32_t rank = cluster_ctarank();
     const int64_t tok0 = static_cast<int64_t>(cluster_id_x()) * kRouteClusterTokens;
     const int tb = static_cast<int>(n_tokens - tok0 < kRouteClusterTokens ? n_tokens - tok0
@@ -280,6 +286,9 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(
     // HS is a multiple of 4 and the slice starts on a 16-byte boundary of
     // each weight row when H % 4 == 0 (the launcher's condition)
     const int n4 = hs >> 2;
+    // launched as a programmatic dependent: the router weights (written by
+    // no kernel) start loading before pdl_wait, the token rows after it
+    pdl_launch_dependents();
     if (stage_w) {
         // the slice of every router row, all in flight at once (one memory
         // latency instead of one per expert a warp handles)
@@ -289,9 +298,30 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(
             if (c < n4) cp_async16_route(ws + e * HS + 4 * c, wr + static_cast<int64_t>(e) * H + h0 + 4 * c);
         }
     }
-    for (int i = tid; i < tb * HS; i += 256) {
-        const int t = i / HS, h = i - t * HS;
-        xs[i] = h < hs ? ElemIO<T>::load(x, (tok0 + t) * H + h0 + h) : 0.f;
+    pdl_wait();
+    if (vec_x) {
+        // the tokens' slices in 16-byte chunks, all in flight at once (H and
+        // HS are multiples of the chunk, so the slice is whole chunks); the
+        // columns past H read as zero
+        constexpr int EPC = 16 / static_cast<int>(sizeof(T));
+        const int cpr = HS / EPC, valid = hs / EPC;
+        for (int i = tid; i < tb * cpr; i += 256) {
+            const int t = i / cpr, c = i - t * cpr;
+            T* dst = xb + t * HS + c * EPC;
+            if (c < valid)
+                cp_async16_route(dst, x + (tok0 + t) * H + h0 + c * EPC);
+            else
+                *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
+        if (sizeof(T) != 4)
+            for (int i = tid; i < tb * HS; i += 256) xs[i] = ElemIO<T>::load(xb, i);
+    } else {
+        for (int i = tid; i < tb * HS; i += 256) {
+            const int t = i / HS, h = i - t * HS;
+            xs[i] = h < hs ? ElemIO<T>::load(x, (tok0 + t) * H + h0 + h) : 0.f;
+        }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
@@ -300,20 +330,33 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(
         // (points into xs when the slice is not staged, so that even a
         // speculated load stays inside the allocation)
         const float4* wsv = reinterpret_cast<const float4*>(stage_w ? ws + e * HS : xs);
-        for (int t = 0; t < tb; ++t) {
-            const float4* xv = reinterpret_cast<const float4*>(xs + t * HS);
-            float acc = 0.f;
-            for (int i = lane; i < n4; i += 32) {
-                const float4 a = stage_w ? wsv[i] : __ldg(wg + i);
-                const float4 b = xv[i];
-                acc = fmaf(a.x, b.x, acc);
-                acc = fmaf(a.y, b.y, acc);
-                acc = fmaf(a.z, b.z, acc);
-                acc = fmaf(a.w, b.w, acc);
-            }
+        // one pass over the expert's slice for all the block's tokens (a
+        // weight chunk is read once and used tb times); per logit the lane
+        // order of the products and the butterfly are those of one token
+        float acc[TBM];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (lane == 0) part[t * E + e] = acc;
+        for (int t = 0; t < TBM; ++t) acc[t] = 0.f;
+        for (int i = lane; i < n4; i += 32) {
+            const float4 a = stage_w ? wsv[i] : __ldg(wg + i);
+#pragma unroll
+            for (int t = 0; t < TBM; ++t) {
+                if (TBM == 1 || t < tb) {
+                    const float4 b = reinterpret_cast<const float4*>(xs + t * HS)[i];
+                    acc[t] = fmaf(a.x, b.x, acc[t]);
+                    acc[t] = fmaf(a.y, b.y, acc[t]);
+                    acc[t] = fmaf(a.z, b.z, acc[t]);
+                    acc[t] = fmaf(a.w, b.w, acc[t]);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < TBM; ++t) {
+            if (TBM == 1 || t < tb) {
+                float v = acc[t];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0) part[t * E + e] = v;
+            }
         }
     }
     cluster_sync();
@@ -346,7 +389,8 @@ cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float*
                                  const float* bias, float* logits, int32_t* idx, float* w,
                                  cudaStream_t st) {
     if (s.H % 4 != 0 || s.T > 64 * kRouteClusterTokens) return cudaErrorNotSupported;
-    const int HS = ((s.H + kRouteCluster - 1) / kRouteCluster + 3) & ~3;
+    // slices of whole 16-byte chunks of the token rows (8 bf16 or 4 floats)
+    const int HS = ((s.H + kRouteCluster - 1) / kRouteCluster + 7) & ~7;
     size_t smem = sizeof(float) * (((kRouteClusterTokens * s.E + 3) & ~3) +
                                    static_cast<size_t>(kRouteClusterTokens) * HS);
     if (smem > 96 * 1024 || static_cast<size_t>(kRouteClusterTokens) * s.E >
@@ -356,33 +400,43 @@ cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float*
     const size_t w_bytes = sizeof(float) * static_cast<size_t>(s.E) * HS;
     const int stage_w = smem + w_bytes <= 160 * 1024 ? 1 : 0;
     if (stage_w) smem += w_bytes;
+    // bf16 rows load in 16-byte chunks into a staging area behind the slice
+    // (float rows straight into theirs) when every row starts on 16 bytes
+    const int vec_x = (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
+                      (s.dtype == MOE_BF16 ? s.H % 8 == 0 : true);
+    if (vec_x && s.dtype == MOE_BF16) smem += 2 * static_cast<size_t>(kRouteClusterTokens) * HS;
     const int blocks = static_cast<int>((s.T + kRouteClusterTokens - 1) / kRouteClusterTokens);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks * kRouteCluster));
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kRouteCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (s.dtype == MOE_BF16) {
-        auto kern = route_cluster_kernel<__nv_bfloat16>;
+        auto kern = s.T == 1 ? route_cluster_kernel<__nv_bfloat16, 1>
+                             : route_cluster_kernel<__nv_bfloat16, kRouteClusterTokens>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(x), wr, bias, logits,
-                                  idx, w, static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w);
+                                  idx, w, static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w,
+                                  vec_x);
     }
-    auto kern = route_cluster_kernel<float>;
+    auto kern = s.T == 1 ? route_cluster_kernel<float, 1>
+                         : route_cluster_kernel<float, kRouteClusterTokens>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const float*>(x), wr, bias, logits, idx, w,
-                              static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w);
+                              static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w, vec_x);
 }
 
 cudaError_t launch_route_small(const moe_shape& s, const void* x, const float* wr,
