@@ -409,7 +409,6 @@ __global__ void __launch_bounds__(bwd::THREADS, 1) grouped_gemm_bwd(
             if (MODE == kWgrad) {
                 const int M = c.routed ? p.M_routed : p.M_shared;
                 const int eidx = c.routed ? c.g : c.g - p.E;
-                const int m = c.m0 + r_in_tile;
                 const bool has_k = num_kb(c) > 0;
                 // the warp's 32 rows x 16 columns are staged in shared memory
                 // (row = lane, 64-byte swizzle: 16-byte chunk q of row r at
