@@ -353,12 +353,11 @@ class Workload:
                         stream=stream)
 
     def step(self, stream, fwd_start=None, fwd_end=None):
-        """route -> permute -> forward -> combine, with events around the forward."""
+        """route + permute -> forward -> combine, with events around the forward."""
         moe, s, L = self.moe, self.shape, self.layer
         b = L.buf
-        idx, w, _ = moe.route(s, self.x, L.w_router, L.router_bias, out=b, w_split=L.w_split,
-                              err_flag=L.err_flag, stream=stream)
-        moe.permute(s, idx, L.workspace, L.err_flag, out=b, stream=stream)
+        moe.route_permute(s, self.x, L.w_router, L.router_bias, L.workspace, L.err_flag, out=b,
+                          stream=stream, w_split=L.w_split)
         if fwd_start is not None:
             fwd_start.record(stream)
         self.forward(stream)

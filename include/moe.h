@@ -107,10 +107,11 @@ MOE_API moe_status moe_workspace_size(const moe_shape* shape, size_t* bytes);
  *                       descending order; equal logits go to the lower index
  *   topk_w      [T, k]  float32 output: softmax over the k selected logits
  *   err_flag    [1]     int32 device word, or NULL (see conventions)
- * Logits accumulate in float32.  Up to 256 tokens run one CTA per token on the
- * CUDA cores; more tokens with bf16 x and E <= 64 run on the tensor cores,
- * the float32 weight split into three bf16 terms (exact to one float32 ulp);
- * anything else runs on the CUDA cores. */
+ * Logits accumulate in float32.  Up to 256 tokens run on the CUDA cores, a
+ * cluster of 8 CTAs per 16 tokens splitting H (one CTA per token where that
+ * does not fit in shared memory); more tokens with bf16 x and E <= 64 run on
+ * the tensor cores, the float32 weight split into three bf16 terms (exact to
+ * one float32 ulp); anything else runs on the CUDA cores. */
 MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const float* w_router,
                              const float* router_bias, float* logits, int32_t* topk_idx,
                              float* topk_w, int32_t* err_flag, void* stream);
@@ -197,6 +198,20 @@ MOE_API moe_status moe_route_noaux_tc(const moe_shape* shape, int32_t n_group,
 MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* err_flag,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* moe_route_split followed by moe_permute, in one call: the outputs of both,
+ * equal to what the two calls write (the same logits, selection, weights and
+ * plan).  Arguments as the two calls; `workspace` as moe_permute's (checked
+ * in every case).  For decode batches of up to 16 tokens with the cluster
+ * router (H % 4 == 0, H <= 32768, a 16-byte aligned w_router) it is ONE
+ * launch: the CTA that selects the experts of all the tokens also builds the
+ * plan.  Otherwise it makes the two calls. */
+MOE_API moe_status moe_route_permute(const moe_shape* shape, const void* x,
+                                     const float* w_router, const void* w_split,
+                                     const float* router_bias, float* logits, int32_t* topk_idx,
+                                     float* topk_w, int32_t* counts, int32_t* offsets,
+                                     int32_t* perm, int32_t* inv, int32_t* err_flag,
+                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* moe_permute for callers that cannot allocate device memory: for example a
  * plugin whose host framework owns every device allocation and hands it only

@@ -16,7 +16,9 @@ cudaError_t launch_route_tc_split(const moe_shape&, const void*, const void*, co
 cudaError_t launch_route_small(const moe_shape&, const void*, const float*, const float*, float*,
                                int32_t*, float*, cudaStream_t);
 cudaError_t launch_route_cluster(const moe_shape&, const void*, const float*, const float*, float*,
-                               int32_t*, float*, cudaStream_t);
+                                 int32_t*, float*, int32_t*, int32_t*, int32_t*, int32_t*,
+                                 cudaStream_t);
+constexpr int64_t kRoutePlanTokens = 16;   // tokens of one cluster block (route.cu)
 size_t permute_workspace_bytes(const moe_shape&);
 cudaError_t launch_permute(const moe_shape&, const int32_t*, int32_t*, int32_t*, int32_t*,
                            int32_t*, int32_t*, void*, cudaStream_t);
@@ -205,7 +207,8 @@ moe_status moe_route(const moe_shape* shape, const void* x, const float* w_route
     // tensor cores; else CUDA cores
     if (shape->T <= 256 && shape->H <= 32768 && aligned16(w_router)) {
         const cudaError_t e = moe::launch_route_cluster(*shape, x, w_router, router_bias, logits,
-                                                        topk_idx, topk_w, cs);
+                                                        topk_idx, topk_w, nullptr, nullptr,
+                                                        nullptr, nullptr, cs);
         if (e != cudaErrorNotSupported) return cuda_status(e);
         return cuda_status(moe::launch_route_small(*shape, x, w_router, router_bias, logits,
                                                    topk_idx, topk_w, cs));
@@ -289,6 +292,33 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t*
     void* blk = static_cast<char*>(workspace) + w.permute_off;
     return cuda_status(moe::launch_permute(*shape, topk_idx, counts, offsets, perm, inv, err_flag,
                                            blk, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_route_permute(const moe_shape* shape, const void* x, const float* w_router,
+                             const void* w_split, const float* router_bias, float* logits,
+                             int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                             int32_t* perm, int32_t* inv, int32_t* err_flag, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (shape->T > 0 && (!x || !w_router || !topk_idx || !topk_w || !perm || !inv))
+        return MOE_ERR_INVALID_ARG;
+    const Workspace w = layout(*shape);
+    if (w.total > 0 && (!workspace || workspace_bytes < w.total)) return MOE_ERR_WORKSPACE;
+    // one token block: the cluster router writes the plan too
+    if (shape->T > 0 && shape->T <= moe::kRoutePlanTokens && shape->H <= 32768 &&
+        aligned16(w_router)) {
+        const cudaError_t e = moe::launch_route_cluster(*shape, x, w_router, router_bias, logits,
+                                                        topk_idx, topk_w, counts, offsets, perm,
+                                                        inv, static_cast<cudaStream_t>(stream));
+        if (e != cudaErrorNotSupported) return cuda_status(e);
+    }
+    st = moe_route_split(shape, x, w_router, w_split, router_bias, logits, topk_idx, topk_w,
+                         err_flag, stream);
+    if (st != MOE_OK) return st;
+    return moe_permute(shape, topk_idx, counts, offsets, perm, inv, err_flag, workspace,
+                       workspace_bytes, stream);
 }
 
 }  // extern "C"

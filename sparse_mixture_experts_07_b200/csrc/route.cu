@@ -139,7 +139,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
 __device__ __forceinline__ void select_topk_warp(const float* lg, int E, int k, int64_t tok,
                                                  float* __restrict__ logits,
                                                  int32_t* __restrict__ topk_idx,
-                                                 float* __restrict__ topk_w) {
+                                                 float* __restrict__ topk_w,
+                                                 int32_t* sel_copy = nullptr) {
     const int lane = threadIdx.x & 31;
     if (logits)
         for (int e = lane; e < E; e += 32) logits[tok * E + e] = lg[e];
@@ -174,6 +175,7 @@ __device__ __forceinline__ void select_topk_warp(const float* lg, int E, int k, 
         for (int r = 0; r < k; ++r) {
             topk_idx[tok * k + r] = sel_e[r];
             topk_w[tok * k + r] = expf(sel_v[r] - sel_v[0]) / den;
+            if (sel_copy) sel_copy[r] = sel_e[r];   // (shared memory, for the plan)
         }
     }
 }
@@ -268,8 +270,15 @@ template <typename T, int TBM>
 __global__ void __launch_bounds__(256) route_cluster_kernel(
     const T* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias,
     float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    int64_t n_tokens, int H, int E, int k, int HS, int stage_w, int vec_x) {
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv, int64_t n_tokens, int H, int E, int k, int HS, int stage_w,
+    int vec_x) {
     extern __shared__ float4 smem_f4[];
+    // the selected experts of the block's slots and the plan's counts and
+    // offsets, when this launch also builds the dispatch plan (perm != NULL)
+    __shared__ int32_t plan_idx[kRouteClusterTokens * kMaxK];
+    __shared__ int32_t plan_cnt[kMaxExperts];
+    __shared__ int32_t plan_off[kMaxExperts];
     float* part = reinterpret_cast<float*>(smem_f4);              // [TB][E] partial logits
     float* xs = part + ((kRouteClusterTokens * E + 3) & ~3);      // [TB][HS]
     float* ws = xs + kRouteClusterTokens * HS;                    // [E][HS] if stage_w
@@ -378,17 +387,71 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(
         }
         __syncthreads();
         for (int t = warp; t < tb; t += 8)
-            select_topk_warp(lg + t * E, E, k, tok0 + t, logits, topk_idx, topk_w);
+            select_topk_warp(lg + t * E, E, k, tok0 + t, logits, topk_idx, topk_w,
+                             perm ? plan_idx + t * k : nullptr);
+        if (perm) {
+            // the one block holds every token: its dispatch plan as
+            // moe_permute defines it (counts, their exclusive prefix sum,
+            // slots in (expert, slot id) order), built here in one pass
+            __syncthreads();
+            const int n = tb * k;
+            for (int e = tid; e < E; e += 256) {
+                int c = 0;
+                for (int q = 0; q < n; ++q) c += plan_idx[q] == e;
+                plan_cnt[e] = c;
+                counts[e] = c;
+            }
+            __syncthreads();
+            if (warp == 0) {
+                const int per = (E + 31) / 32;      // consecutive experts per lane
+                int own = 0;
+                for (int j = 0; j < per; ++j) {
+                    const int e = lane * per + j;
+                    if (e < E) own += plan_cnt[e];
+                }
+                int incl = own;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                int run = incl - own;
+                for (int j = 0; j < per; ++j) {
+                    const int e = lane * per + j;
+                    if (e < E) {
+                        plan_off[e] = run;
+                        offsets[e] = run;
+                        run += plan_cnt[e];
+                    }
+                }
+                if (lane == 31) offsets[E] = incl;
+            }
+            __syncthreads();
+            for (int q = tid; q < n; q += 256) {
+                const int e = plan_idx[q];
+                int before = 0;
+                for (int q2 = 0; q2 < q; ++q2) before += plan_idx[q2] == e;
+                const int p = plan_off[e] + before;
+                perm[p] = q;
+                inv[q] = p;
+            }
+        }
     }
     cluster_sync();
 }
 
 // The cluster kernel when its shared memory fits (decode batches); returns
-// cudaErrorNotSupported otherwise so that the caller takes route_small.
+// cudaErrorNotSupported otherwise so that the caller takes route_small.  With
+// `perm` non-NULL it also writes the dispatch plan (counts, offsets, perm,
+// inv), which needs every token in one block: more than kRouteClusterTokens
+// tokens return cudaErrorNotSupported.
 cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float* wr,
                                  const float* bias, float* logits, int32_t* idx, float* w,
+                                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                                  cudaStream_t st) {
     if (s.H % 4 != 0 || s.T > 64 * kRouteClusterTokens) return cudaErrorNotSupported;
+    if (perm && (s.T > kRouteClusterTokens || s.k > kMaxK || s.E > kMaxExperts))
+        return cudaErrorNotSupported;
     // slices of whole 16-byte chunks of the token rows (8 bf16 or 4 floats)
     const int HS = ((s.H + kRouteCluster - 1) / kRouteCluster + 7) & ~7;
     size_t smem = sizeof(float) * (((kRouteClusterTokens * s.E + 3) & ~3) +
@@ -427,8 +490,8 @@ cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float*
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(x), wr, bias, logits,
-                                  idx, w, static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w,
-                                  vec_x);
+                                  idx, w, counts, offsets, perm, inv, static_cast<int64_t>(s.T),
+                                  s.H, s.E, s.k, HS, stage_w, vec_x);
     }
     auto kern = s.T == 1 ? route_cluster_kernel<float, 1>
                          : route_cluster_kernel<float, kRouteClusterTokens>;
@@ -436,7 +499,8 @@ cudaError_t launch_route_cluster(const moe_shape& s, const void* x, const float*
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const float*>(x), wr, bias, logits, idx, w,
-                              static_cast<int64_t>(s.T), s.H, s.E, s.k, HS, stage_w, vec_x);
+                              counts, offsets, perm, inv, static_cast<int64_t>(s.T), s.H, s.E, s.k,
+                              HS, stage_w, vec_x);
 }
 
 cudaError_t launch_route_small(const moe_shape& s, const void* x, const float* wr,

@@ -58,6 +58,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_workspace_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
     lib.moe_route.argtypes = [S, P, P, P, P, P, P, P, P]
     lib.moe_permute.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.moe_route_permute.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                      ctypes.c_size_t, P]
     lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_combine.argtypes = [S, P, P, P, P]
     lib.moe_router_split_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
@@ -208,6 +210,32 @@ def permute(shape: Shape, topk_idx, workspace, err_flag, out=None, stream=None):
                            _ptr(perm), _ptr(inv), _ptr(err_flag), _ptr(workspace),
                            workspace.numel(), _stream(stream)), "moe_permute")
     return counts, offsets, perm, inv
+
+
+def route_permute(shape: Shape, x, w_router, router_bias, workspace, err_flag, out=None,
+                  logits=False, stream=None, w_split=None):
+    """route then permute in one call (moe_route_permute; one launch for up to
+    16 tokens): (topk_idx, topk_w, logits or None, counts, offsets, perm, inv)."""
+    lib = load_library()
+    dev = x.device
+    n = shape.T * shape.k
+    if out:
+        idx, w = out["topk_idx"], out["topk_w"]
+        counts, offsets, perm, inv = out["counts"], out["offsets"], out["perm"], out["inv"]
+    else:
+        idx = torch.empty(shape.T, shape.k, dtype=torch.int32, device=dev)
+        w = torch.empty(shape.T, shape.k, dtype=torch.float32, device=dev)
+        counts = torch.empty(shape.E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(shape.E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(n, dtype=torch.int32, device=dev)
+        inv = torch.empty(n, dtype=torch.int32, device=dev)
+    lg = torch.empty(shape.T, shape.E, dtype=torch.float32, device=dev) if logits else None
+    _check(lib.moe_route_permute(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(w_split),
+                                 _ptr(router_bias), _ptr(lg), _ptr(idx), _ptr(w), _ptr(counts),
+                                 _ptr(offsets), _ptr(perm), _ptr(inv), _ptr(err_flag),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_route_permute")
+    return idx, w, lg, counts, offsets, perm, inv
 
 
 def forward(shape: Shape, x, offsets, perm, topk_w, gate_up, down, sh_gate_up, sh_down,
@@ -401,11 +429,12 @@ class MoELayer:
                                        self.routing[2], out=b, logits=b["logits"],
                                        stream=stream, err_flag=self.err_flag,
                                        w_split=self.w_split)
+            counts, offsets, perm, inv = permute(s, idx, self.workspace, self.err_flag, out=b,
+                                                 stream=stream)
         else:
-            idx, w, _ = route(s, x, self.w_router, self.router_bias, out=b, stream=stream,
-                              err_flag=self.err_flag, w_split=self.w_split)
-        counts, offsets, perm, inv = permute(s, idx, self.workspace, self.err_flag, out=b,
-                                             stream=stream)
+            idx, w, _, counts, offsets, perm, inv = route_permute(
+                s, x, self.w_router, self.router_bias, self.workspace, self.err_flag, out=b,
+                stream=stream, w_split=self.w_split)
         if self.mxfp4 is not None:
             forward_mxfp4(s, x, offsets, perm, w, self.mxfp4, self.workspace, self.err_flag,
                           y_slots=b["y_slots"], stream=stream)

@@ -91,6 +91,12 @@ def test_null_pointers_rejected_before_launch(lib):
                            1 << 30, None) == 1
     assert lib.moe_combine(ctypes.byref(s), None, p, p, None) == 1
     assert lib.moe_route(None, p, p, None, None, p, p, None, None) == 1
+    # moe_route_permute: x, w_router, topk_idx, topk_w, counts, offsets, perm, inv
+    args = [p, p, None, None, None, p, p, p, p, p, p, None, p, 1 << 30, None]
+    for i in (0, 1, 5, 6, 7, 8, 9, 10):
+        a = list(args)
+        a[i] = None
+        assert lib.moe_route_permute(ctypes.byref(s), *a) == 1, i
 
 
 def test_small_workspace_rejected(lib):
@@ -101,6 +107,9 @@ def test_small_workspace_rejected(lib):
     assert lib.moe_permute(ctypes.byref(s), p, p, p, p, p, None, None, need, None) == 3
     assert lib.moe_forward(ctypes.byref(s), p, p, p, p, p, p, None, None, p, None, p,
                            need - 1, None) == 3
+    for ws, n in ((p, need - 1), (None, need)):
+        assert lib.moe_route_permute(ctypes.byref(s), p, p, None, None, None, p, p, p, p, p, p,
+                                     None, ws, n, None) == 3
 
 
 def test_misaligned_bf16_pointers_rejected(lib):
