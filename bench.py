@@ -38,9 +38,9 @@ L2_BYTES = 126 * 1024 * 1024
 # kernels, from one ncu capture, keyed by workload; valid only while the GEMM
 # source is unchanged (sha256 of the file, first 16 hex digits).
 TRAFFIC = {
-    # profiles/traffic_mixtral.md, the later of two captures (the first read
-    # 4.053 GB): gather 0.053 + GEMM 1 2.758 + GEMM 2 1.490 GB
-    "mixtral": {"bytes": 4.301e9, "file": "gemm_sm100_pair.cu", "sha": "1d599c5a5dbfdc6f"},
+    # profiles/traffic_mixtral.md, the capture of this GEMM source (an earlier
+    # one read 4.053 GB): gather 0.053 + GEMM 1 2.758 + GEMM 2 1.490 GB
+    "mixtral": {"bytes": 4.301e9, "file": "gemm_sm100_pair.cu", "sha": "907865b03f8a6821"},
 }
 
 
