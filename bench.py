@@ -345,7 +345,11 @@ class Workload:
         """The moe_forward region alone, on the plan the last step left in the buffers."""
         moe, s, L = self.moe, self.shape, self.layer
         b = L.buf
-        if self.mx is not None:
+        if L.mx_prepared is not None:
+            moe.forward_mxfp4_prepared(s, self.x, b["offsets"], b["perm"], b["topk_w"], self.mx,
+                                       L.mx_prepared, L.workspace, L.err_flag,
+                                       y_slots=b["y_slots"], stream=stream)
+        elif self.mx is not None:
             moe.forward_mxfp4(s, self.x, b["offsets"], b["perm"], b["topk_w"], self.mx,
                               L.workspace, L.err_flag, y_slots=b["y_slots"], stream=stream)
         else:
@@ -372,6 +376,7 @@ class Workload:
 EXTRA_WORKLOADS = [
     ("phimoe_decode1", "bf16"), ("phimoe_decode8", "bf16"), ("phimoe_decode64", "bf16"),
     ("phimoe_decode1", "mxfp4"), ("phimoe_decode8", "mxfp4"), ("phimoe_decode64", "mxfp4"),
+    ("gptoss_decode1", "mxfp4"), ("gptoss_decode8", "mxfp4"),
     ("phimoe_prefill", "bf16"), ("gptoss", "bf16"), ("dsv3", "bf16"),
 ]
 

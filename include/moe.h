@@ -291,6 +291,45 @@ MOE_API moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x,
                                      const uint8_t* down_s, void* y_slots, int32_t* err_flag,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* The MXFP4 weights prepared once, at load time, for the block-scaled
+ * tensor-core kernel ("Mixture of Experts in Transformers", WeightConverter
+ * section: such conversions belong to the weight-loading pipeline):
+ *   - the E8M0 scales re-laid out per (expert, tile of 128 weight rows,
+ *     K-group of 128 weights) as one 512-byte block in the order the kernel
+ *     copies them into tensor memory, so that a K-group takes one bulk copy
+ *     instead of 128 per-row 4-byte reads (GEMM 1 tiles: 64 gate rows and
+ *     the 64 up rows of the same columns; rows past an expert's and blocks
+ *     past K/32 hold 127, 2^0);
+ *   - when H (gate_up) or I (down) is not a multiple of 128, a copy of those
+ *     codes with each row padded by zero codes to a multiple of 128 weights
+ *     (the tensor maps that unpack 4-bit codes take whole 128-weight groups).
+ *
+ * moe_mxfp4_prepared_size writes to *bytes the size of the prepared array for
+ * `shape`, or 0 when H or I is not a multiple of 64.
+ *
+ * moe_mxfp4_prepare fills `prepared` (16-byte aligned, caller-owned) from the
+ * raw arrays of moe_forward_mxfp4; MOE_ERR_UNSUPPORTED when the size is 0 or
+ * a pointer is misaligned, MOE_ERR_WORKSPACE when prepared_bytes is too small.
+ *
+ * moe_forward_mxfp4_prepared is moe_forward_mxfp4 on the tensor cores with
+ * the prepared array in place of the scales, for H and I multiples of 64
+ * (gpt-oss: 2880) as well as 128; gate_up_q and down_q are still the raw
+ * codes (read where K is a multiple of 128).  x, the codes, `prepared`,
+ * y_slots and the workspace 16-byte aligned, the codes 32-byte aligned;
+ * otherwise MOE_ERR_UNSUPPORTED.  Arithmetic as moe_forward_mxfp4's
+ * tensor-core kernel. */
+MOE_API moe_status moe_mxfp4_prepared_size(const moe_shape* shape, size_t* bytes);
+MOE_API moe_status moe_mxfp4_prepare(const moe_shape* shape, const uint8_t* gate_up_q,
+                                     const uint8_t* gate_up_s, const uint8_t* down_q,
+                                     const uint8_t* down_s, void* prepared,
+                                     size_t prepared_bytes, void* stream);
+MOE_API moe_status moe_forward_mxfp4_prepared(const moe_shape* shape, const void* x,
+                                              const int32_t* offsets, const int32_t* perm,
+                                              const float* topk_w, const uint8_t* gate_up_q,
+                                              const uint8_t* down_q, const void* prepared,
+                                              void* y_slots, int32_t* err_flag, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
 /* Combine ("Mixture of Experts in Transformers", expert backends: gather and
  * reorder the results).  y[t] = sum_j y_slots[inv[t*k+j]]
  *                               + sum_s y_slots[T*k + s*T + t],

@@ -117,8 +117,10 @@ struct TcGeo {
 
 struct MxTcParams {
     const int32_t* offsets;     // [E+1]
-    const uint8_t* w_scales;    // [E * wrows, nblk] E8M0 of the weights
-    const uint8_t* act_sf;      // [2 * SP, nblk] E8M0 of the activation planes (hi, then lo)
+    const uint8_t* w_scales;    // [E * wrows, K/32] E8M0 of the weights (K a multiple of 128)
+    const uint8_t* w_tiled;     // or: the weights' E8M0 in tensor-memory order (mx_tc_prepare)
+    const uint8_t* act_sf;      // [2 * SP, sf_stride] E8M0 of the activation planes (hi, then lo)
+    int sf_stride;              // bytes per activation scale row: 4 per K-group
     float* part;                // [splits][S][n_out] fp32 partial sums
     int32_t* ctl;               // ctl[0]: splits used (written by CTA 0)
     int32_t* err_flag;
@@ -192,7 +194,24 @@ __device__ __forceinline__ void cp_async_arrive_noinc_tc(uint64_t* bar) {
                  : "memory");
 }
 
-// TMA tile loads of 4 and 5 dimensions (coordinates innermost first).
+// TMA tile loads of 3 and 4 dimensions (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+// `bytes` (a multiple of 16) from a 16-byte aligned global address into this
+// CTA's shared memory, counted on bar's transaction bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
     asm volatile(
@@ -201,17 +220,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
-__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3,
-                                            int32_t c4) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
-        "r"(c4)
-        : "memory");
-}
-
 // Splits of the contraction, in whole stages of kgs K-groups: the count s <=
 // MAX_SPLITS that minimises the bytes the busiest CTA moves, i.e. the waves
 // of items, ceil(units s / grid), times the stages of an item, plus the
@@ -242,19 +250,25 @@ __host__ __device__ inline int mx_tc_splits(int units, int grid, int n_kg, int k
     return best;
 }
 
-// map_w: the packed codes as a 5D tensor (128 codes of a K-group, R1 rows,
-// R2 row blocks, E experts, K/128 K-groups) so that one box brings KGS whole
-// K-groups of a 128-row tile: per row KGS x 64 contiguous bytes of memory.
+// map_w: the packed codes as a 4D tensor (K codes, R1 rows, R2 row blocks, E
+// experts) so that one box brings a K-group of a 128-row tile: per row 64
+// contiguous bytes of memory; codes past K and row blocks past R2 read as
+// zero.
 //   GEMM 1: R1 = I (gate row), R2 = 2 (gate, up): box rows (mt*64.., 0..1)
 //   GEMM 2: R1 = 64, R2 = H/64: box rows (0..63, 2mt..2mt+1)
-// map_act: the E4M3 planes as a 4D tensor (128 bytes of a K-group, SP rows,
-// 2 planes, K/128 K-groups): box (CH rows, both planes, KGS K-groups).
-template <int KIND, int CH, int KGS, int CPS>
+// map_act: the E4M3 planes as a 3D tensor (K bytes, SP rows, 2 planes): box
+// (128 bytes of a K-group, CH rows, both planes).
+// TILED: the weight scales come as one 512-byte atom per (expert, tile,
+// K-group), prepared once (mx_tc_prepare) in the order tensor memory takes
+// them, and load with one bulk copy; otherwise (K a multiple of 128) each
+// lane copies 4 scale words of the raw [rows, K/32] array.
+template <int KIND, int CH, int KGS, int CPS, bool TILED>
 __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_act,
     const MxTcParams p) {
     using G = TcGeo<CH, KGS, CPS>;
     using namespace mxtc;
+    static_assert(KGS == 1, "the tensor maps bring one K-group per box");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ MxUnits act;
     __shared__ uint32_t tmem_base_sh;
@@ -269,8 +283,9 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
     uint64_t* drain = tempty + 2;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nblk = p.K / 32;
-    const int n_kg = p.K / KG;                  // K-groups of a whole contraction
+    const int nblk = p.K / 32;                  // raw scale row (not TILED: K % 128 == 0)
+    const int n_kg = (p.K + KG - 1) / KG;       // K-groups of a whole contraction (last one
+                                                // partial when K % 128 != 0: zero-filled)
 
     // launched as a programmatic dependent: barriers, descriptor prefetch and
     // tensor memory are set up while the previous kernel finishes; global
@@ -348,8 +363,13 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
             for (int j = 0; j < 4; ++j) {
                 const int w = 32 * j + lane;
                 const int m = (w >> 2) + 32 * (w & 3);
-                wsrc[j] = p.w_scales + (h0 + (m / HALF_ROWS) * hstride + (m % HALF_ROWS)) * nblk;
+                wsrc[j] = TILED ? nullptr
+                                : p.w_scales + (h0 + (m / HALF_ROWS) * hstride + (m % HALF_ROWS)) * nblk;
             }
+            // TILED: this tile's scale atoms, one per K-group
+            const uint8_t* tsrc = TILED ? p.w_tiled + (static_cast<int64_t>(grp) * p.mtiles + mt) *
+                                                         n_kg * SF_ATOM
+                                        : nullptr;
             for (int kg = kg0; kg < kg1; kg += KGS, ++f) {
                 const int nk = kg1 - kg < KGS ? kg1 - kg : KGS;   // K-groups used in this stage
                 const int slot = f % G::STAGES;
@@ -361,19 +381,22 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
                 uint8_t* sfa = sb + G::B_SMEM;
                 uint8_t* sfb = sfa + KGS * SF_ATOM;
                 if (lane == 0) {
-                    // whole boxes always (K-groups past the tensor are zero
-                    // filled; those past kg1 are loaded but not used)
-                    mbar_arrive_expect_tx(&full[slot], G::TX);
+                    // whole boxes always (codes past K and weight rows past the
+                    // expert's are zero filled)
+                    mbar_arrive_expect_tx(&full[slot], G::TX + (TILED ? SF_ATOM : 0));
                     if (KIND == 0)
-                        tma_load_5d(sa, &map_w, &full[slot], 0, mt * HALF_ROWS, 0, grp, kg);
+                        tma_load_4d(sa, &map_w, &full[slot], kg * KG, mt * HALF_ROWS, 0, grp);
                     else
-                        tma_load_5d(sa, &map_w, &full[slot], 0, 0, 2 * mt, grp, kg);
-                    tma_load_4d(sb, &map_act, &full[slot], 0, brow0, 0, kg);
+                        tma_load_4d(sa, &map_w, &full[slot], kg * KG, 0, 2 * mt, grp);
+                    tma_load_3d(sb, &map_act, &full[slot], kg * KG, brow0, 0);
+                    if (TILED) bulk_load(sfa, tsrc + static_cast<int64_t>(kg) * SF_ATOM, SF_ATOM, &full[slot]);
                 }
                 for (int c = 0; c < nk; ++c) {
+                    if (!TILED) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        cp_async4_tc(sfa + c * SF_ATOM + 4 * (32 * j + lane), wsrc[j] + 4 * (kg + c), 4u);
+                        for (int j = 0; j < 4; ++j)
+                            cp_async4_tc(sfa + c * SF_ATOM + 4 * (32 * j + lane), wsrc[j] + 4 * (kg + c), 4u);
+                    }
 #pragma unroll
                     for (int j = 0; j < (G::N + 31) / 32; ++j) {
                         const int n = lane + 32 * j;
@@ -382,7 +405,8 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
                             const int srow = brow0 + (n - plane * CH);
                             const bool in = srow < p.S;          // rows past the slots: zeros
                             const uint8_t* src = p.act_sf +
-                                (static_cast<int64_t>(plane) * p.SP + (in ? srow : 0)) * nblk + 4 * (kg + c);
+                                (static_cast<int64_t>(plane) * p.SP + (in ? srow : 0)) * p.sf_stride +
+                                4 * (kg + c);
                             cp_async4_tc(sfb + c * SF_ATOM + 16 * lane + 4 * j, src, in ? 4u : 0u);
                         }
                     }
@@ -492,9 +516,10 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
             else
                 n_o = mt * 128 + m;
             float* dst = p.part + (static_cast<int64_t>(sp) * p.S + brow0) * p.n_out + n_o;
+            const bool row_in = KIND == 0 || n_o < p.n_out;   // GEMM 2: tile rows past H
 #pragma unroll
             for (int c = 0; c < CH; ++c)
-                if (c < rows) dst[static_cast<int64_t>(c) * p.n_out] = v[c] + v[CH + c];
+                if (c < rows && row_in) dst[static_cast<int64_t>(c) * p.n_out] = v[c] + v[CH + c];
         }
     }
 
@@ -535,47 +560,60 @@ __device__ __forceinline__ float warp_max_abs(float v) {
 }
 
 // One warp per (slot row, 32-block): writes the value's hi byte to plane 0
-// (row r) and lo byte to plane 1 (row SP + r), and the exponents likewise.
+// (row r) and lo byte to plane 1 (row SP + r), and the exponents likewise
+// (scale rows of sf_stride bytes).
 __device__ __forceinline__ void store_e4m3_pair(float v, int64_t r, int blk, int K, int SP,
-                                                uint8_t* q, uint8_t* sf) {
+                                                int sf_stride, uint8_t* q, uint8_t* sf) {
     const int lane = threadIdx.x & 31;
     const float bmax = warp_max_abs(v);
     uint8_t hi, lo;
     int eh, el;
     e4m3_pair(v, bmax, hi, lo, eh, el);
-    const int nblk = K / 32;
     q[r * K + blk * 32 + lane] = hi;
     q[(SP + r) * K + blk * 32 + lane] = lo;
     if (lane == 0) {
-        sf[r * nblk + blk] = static_cast<uint8_t>(eh + 127);
-        sf[(SP + r) * nblk + blk] = static_cast<uint8_t>(el + 127);
+        sf[r * sf_stride + blk] = static_cast<uint8_t>(eh + 127);
+        sf[(SP + r) * sf_stride + blk] = static_cast<uint8_t>(el + 127);
     }
+}
+
+// Scale bytes of the blocks past K that fill the last K-group (K % 128 != 0):
+// 2^0, a finite factor for codes the tensor map reads as zero.  True when
+// `blk` is such a block (written) or past the row (nothing to do).
+__device__ __forceinline__ bool pad_scale_block(int64_t r, int blk, int K, int SP, int sf_stride,
+                                                uint8_t* sf) {
+    if (blk < K / 32) return false;
+    if (blk < sf_stride && (threadIdx.x & 31) == 0) {
+        sf[r * sf_stride + blk] = 127;
+        sf[(SP + r) * sf_stride + blk] = 127;
+    }
+    return true;
 }
 
 // GEMM 1 operand B: x[perm[r] / k] of every sorted slot row r.
 __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_prep_x_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int k, int K, int SP,
-    uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    int sf_stride, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
     pdl_launch_dependents();
     pdl_wait();
     const int r = blockIdx.y;
     const int blk = blockIdx.x * (mxtc::PREP_THREADS / 32) + (threadIdx.x >> 5);
-    if (blk >= K / 32) return;
+    if (pad_scale_block(r, blk, K, SP, sf_stride, sf)) return;
     const int64_t tok = perm[r] / k;
     const float v = __bfloat162float(x[tok * K + blk * 32 + (threadIdx.x & 31)]);
-    store_e4m3_pair(v, r, blk, K, SP, q, sf);
+    store_e4m3_pair(v, r, blk, K, SP, sf_stride, q, sf);
 }
 
 // GEMM 1 epilogue: gate and up summed over the splits in order, h =
 // SiLU(gate) * up rounded to bf16, then quantised as GEMM 2's operand B.
 __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_swiglu_kernel(
     const float* __restrict__ part, const int32_t* __restrict__ ctl, int S, int I, int SP,
-    uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    int sf_stride, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
     pdl_launch_dependents();
     pdl_wait();
     const int r = blockIdx.y;
     const int blk = blockIdx.x * (mxtc::PREP_THREADS / 32) + (threadIdx.x >> 5);
-    if (blk >= I / 32) return;
+    if (pad_scale_block(r, blk, I, SP, sf_stride, sf)) return;
     const int i = blk * 32 + (threadIdx.x & 31);
     const int splits = ctl[0];
     float g = 0.f, u = 0.f;
@@ -585,7 +623,7 @@ __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_swiglu_kernel(
         u += row[I + i];
     }
     const float h = __bfloat162float(__float2bfloat16_rn(g / (1.f + __expf(-g)) * u));
-    store_e4m3_pair(h, r, blk, I, SP, q, sf);
+    store_e4m3_pair(h, r, blk, I, SP, sf_stride, q, sf);
 }
 
 // GEMM 2 epilogue: y_slots[r] = routed_scale * topk_w[perm[r]] * sum over splits.
@@ -608,44 +646,38 @@ __global__ void __launch_bounds__(256) mx_tc_down_out_kernel(
 // ------------------------------------------------------------------ launcher
 
 // Packed E2M1 codes [E * wrows, K/2 bytes] read as 16U4_ALIGN16B (each 16
-// codes land in 16 bytes of shared memory, 128-byte swizzle) through the 5D
+// codes land in 16 bytes of shared memory, 128-byte swizzle) through the 4D
 // view described above the kernel; box (128 codes, 64 rows, 2 row blocks, 1
-// expert, kgs K-groups).
+// expert).
 static bool make_map_e2m1(CUtensorMap* map, const void* base, int E, int64_t wrows, int64_t K,
-                          int64_t r1, int64_t r2, int64_t r1_rows_stride, int kgs) {
+                          int64_t r1, int64_t r2, int64_t r1_rows_stride) {
     EncodeTiledFn enc = get_encode_fn();
-    if (!enc || E <= 0 || K <= 0 || K % mxtc::KG != 0) return false;
+    if (!enc || E <= 0 || K <= 0 || K % 32 != 0) return false;
     const cuuint64_t row_bytes = static_cast<cuuint64_t>(K / 2);
-    cuuint64_t dims[5] = {static_cast<cuuint64_t>(mxtc::KG), static_cast<cuuint64_t>(r1),
-                          static_cast<cuuint64_t>(r2), static_cast<cuuint64_t>(E),
-                          static_cast<cuuint64_t>(K / mxtc::KG)};
-    cuuint64_t strides[4] = {row_bytes, row_bytes * static_cast<cuuint64_t>(r1_rows_stride),
-                             row_bytes * static_cast<cuuint64_t>(wrows),
-                             static_cast<cuuint64_t>(mxtc::KG / 2)};
-    cuuint32_t box[5] = {static_cast<cuuint32_t>(mxtc::KG), static_cast<cuuint32_t>(mxtc::HALF_ROWS),
-                         2u, 1u, static_cast<cuuint32_t>(kgs)};
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 5, const_cast<void*>(base), dims,
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(r1),
+                          static_cast<cuuint64_t>(r2), static_cast<cuuint64_t>(E)};
+    cuuint64_t strides[3] = {row_bytes, row_bytes * static_cast<cuuint64_t>(r1_rows_stride),
+                             row_bytes * static_cast<cuuint64_t>(wrows)};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(mxtc::KG), static_cast<cuuint32_t>(mxtc::HALF_ROWS),
+                         2u, 1u};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void*>(base), dims,
                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// E4M3 activation planes [2 * SP rows, K bytes] as a 4D tensor (128 bytes of
-// a K-group, SP rows, 2 planes, K/128 K-groups); box (128, ch rows, 2 planes,
-// kgs K-groups), 128-byte swizzle.
-static bool make_map_e4m3(CUtensorMap* map, const void* base, int64_t SP, int64_t K, int ch,
-                          int kgs) {
+// E4M3 activation planes [2 * SP rows, K bytes] as a 3D tensor (K bytes, SP
+// rows, 2 planes); box (128 bytes of a K-group, ch rows, 2 planes), 128-byte
+// swizzle; bytes past K read as zero.
+static bool make_map_e4m3(CUtensorMap* map, const void* base, int64_t SP, int64_t K, int ch) {
     EncodeTiledFn enc = get_encode_fn();
-    if (!enc || SP <= 0 || K <= 0 || K % mxtc::KG != 0) return false;
-    cuuint64_t dims[4] = {static_cast<cuuint64_t>(mxtc::KG), static_cast<cuuint64_t>(SP), 2u,
-                          static_cast<cuuint64_t>(K / mxtc::KG)};
-    cuuint64_t strides[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(SP * K),
-                             static_cast<cuuint64_t>(mxtc::KG)};
-    cuuint32_t box[4] = {static_cast<cuuint32_t>(mxtc::KG), static_cast<cuuint32_t>(ch), 2u,
-                         static_cast<cuuint32_t>(kgs)};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box,
+    if (!enc || SP <= 0 || K <= 0 || K % 32 != 0) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(SP), 2u};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(SP * K)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(mxtc::KG), static_cast<cuuint32_t>(ch), 2u};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -662,45 +694,210 @@ int64_t mx_tc_part_floats(int64_t slots, int H, int I) {
     return rows * cols;
 }
 
-bool mx_tc_supported(const moe_shape& s, const void* gu_q, const void* dn_q) {
-    return s.H % 128 == 0 && s.I % 128 == 0 && s.T >= 1 && s.T <= 64 &&
+// Activation scale rows: 4 bytes per K-group, whole K-groups.
+static int mx_tc_sf_stride(int K) { return (K + mxtc::KG - 1) / mxtc::KG * 4; }
+
+// The prepared weights of the tensor-core path (mx_tc_prepare), in this
+// order, each part 256-byte aligned:
+//   tiled scales, GEMM 1: one SF_ATOM per (expert, I/64 tiles, ceil(H/128)
+//     K-groups); GEMM 2: per (expert, ceil(H/128) tiles, ceil(I/128) K-groups)
+//   when H % 128 != 0: gate_up codes with rows padded by zero codes to a
+//     multiple of 128 weights [E, 2I, Hp/2];  when I % 128 != 0: down codes
+//     likewise [E, H, Ip/2]
+// (the 4-bit unpacking tensor maps take rows of whole 128-weight K-groups
+// only).  0 bytes when the tensor-core kernel cannot take the shape.
+static int64_t align256(int64_t v) { return (v + 255) / 256 * 256; }
+static int64_t round128(int64_t v) { return (v + 127) / 128 * 128; }
+static int64_t mx_tc_tiled_gu_bytes(const moe_shape& s) {
+    return static_cast<int64_t>(mxtc::SF_ATOM) * s.E * (s.I / mxtc::HALF_ROWS) *
+           ((s.H + mxtc::KG - 1) / mxtc::KG);
+}
+static int64_t mx_tc_tiled_dn_bytes(const moe_shape& s) {
+    return static_cast<int64_t>(mxtc::SF_ATOM) * s.E * ((s.H + 127) / 128) *
+           ((s.I + mxtc::KG - 1) / mxtc::KG);
+}
+static int64_t mx_tc_gu_pad_bytes(const moe_shape& s) {
+    return s.H % 128 ? static_cast<int64_t>(s.E) * 2 * s.I * (round128(s.H) / 2) : 0;
+}
+static int64_t mx_tc_dn_pad_bytes(const moe_shape& s) {
+    return s.I % 128 ? static_cast<int64_t>(s.E) * s.H * (round128(s.I) / 2) : 0;
+}
+int64_t mx_tc_prepared_bytes(const moe_shape& s) {
+    if (s.H % 64 != 0 || s.I % 64 != 0 || s.H <= 0 || s.I <= 0) return 0;
+    return align256(mx_tc_tiled_gu_bytes(s)) + align256(mx_tc_tiled_dn_bytes(s)) +
+           align256(mx_tc_gu_pad_bytes(s)) + align256(mx_tc_dn_pad_bytes(s));
+}
+struct MxPrepared {
+    const uint8_t* tiled;        // GEMM 1's atoms, then GEMM 2's at tiled_dn
+    const uint8_t* tiled_dn;
+    const uint8_t* gu_codes;     // padded copies, or NULL (use the caller's codes)
+    const uint8_t* dn_codes;
+};
+static MxPrepared mx_tc_prepared_parts(const moe_shape& s, const void* base) {
+    const uint8_t* b = static_cast<const uint8_t*>(base);
+    MxPrepared m;
+    m.tiled = b;
+    m.tiled_dn = b + align256(mx_tc_tiled_gu_bytes(s));
+    const uint8_t* pads = m.tiled_dn + align256(mx_tc_tiled_dn_bytes(s));
+    m.gu_codes = mx_tc_gu_pad_bytes(s) ? pads : nullptr;
+    m.dn_codes = mx_tc_dn_pad_bytes(s) ? pads + align256(mx_tc_gu_pad_bytes(s)) : nullptr;
+    return m;
+}
+
+// Rows of K/2 code bytes copied into rows of Kp/2 bytes, the rest zero (16-byte
+// vectors: K % 32 == 0, Kp % 128 == 0).
+__global__ void __launch_bounds__(256) mx_tc_pad_codes_kernel(const uint4* __restrict__ src,
+                                                              uint4* __restrict__ dst,
+                                                              int64_t rows, int K, int Kp) {
+    const int vin = K / 32, vout = Kp / 32;      // 16-byte vectors per row
+    const int64_t n = rows * vout;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / vout;
+        const int v = static_cast<int>(i - r * vout);
+        dst[i] = v < vin ? src[r * vin + v] : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// The weight scales of both GEMMs in the order the tensor-core kernel copies
+// them into tensor memory: per (expert, tile, K-group) an atom whose byte
+// 4 w + kb is the scale of tile row (w >> 2) + 32 (w & 3), K-block 4 kg + kb
+// (GEMM 1 tile rows: 64 gate rows, then the 64 up rows of the same columns);
+// rows past the expert's and K-blocks past K/32 hold 127 (2^0, against codes
+// the tensor maps read as zero).  One thread per 4-byte word.
+__global__ void __launch_bounds__(256) mx_tc_tile_scales_kernel(
+    const uint8_t* __restrict__ gu_s, const uint8_t* __restrict__ dn_s,
+    uint32_t* __restrict__ out, int E, int H, int I, int64_t n_gu_words, int64_t n_words) {
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n_words;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const bool gu = idx < n_gu_words;
+        const int64_t j = gu ? idx : idx - n_gu_words;
+        const int K = gu ? H : I;
+        const int nkb = K / 32;
+        const int n_kg = (K + mxtc::KG - 1) / mxtc::KG;
+        const int mtiles = gu ? I / mxtc::HALF_ROWS : (H + 127) / 128;
+        const int w = static_cast<int>(j % 128);
+        const int64_t t = j / 128;
+        const int kg = static_cast<int>(t % n_kg);
+        const int mt = static_cast<int>((t / n_kg) % mtiles);
+        const int e = static_cast<int>(t / (static_cast<int64_t>(n_kg) * mtiles));
+        const int m = (w >> 2) + 32 * (w & 3);
+        int64_t row;          // within the expert
+        bool valid;
+        if (gu) {
+            row = m < mxtc::HALF_ROWS ? static_cast<int64_t>(mt) * mxtc::HALF_ROWS + m
+                                      : I + static_cast<int64_t>(mt) * mxtc::HALF_ROWS + (m - mxtc::HALF_ROWS);
+            valid = true;
+        } else {
+            row = static_cast<int64_t>(mt) * 128 + m;
+            valid = row < H;
+        }
+        const uint8_t* src = (gu ? gu_s + (static_cast<int64_t>(e) * 2 * I + row) * nkb
+                                 : dn_s + (static_cast<int64_t>(e) * H + row) * nkb);
+        uint32_t word = 0;
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+            const int blk = 4 * kg + kb;
+            const uint32_t v = (valid && blk < nkb) ? src[blk] : 127u;
+            word |= v << (8 * kb);
+        }
+        out[idx] = word;
+    }
+}
+
+static int grid_of(int64_t n, int num_sms) {
+    const int64_t want = (n + 255) / 256;
+    return static_cast<int>(want < 8 * num_sms ? (want > 0 ? want : 1) : 8 * num_sms);
+}
+
+// Fills the prepared weights (layout above mx_tc_prepared_bytes).
+cudaError_t launch_mx_tc_prepare(const moe_shape& s, const uint8_t* gu_q, const uint8_t* gu_s,
+                                 const uint8_t* dn_q, const uint8_t* dn_s, void* out, int num_sms,
+                                 cudaStream_t st) {
+    if (mx_tc_prepared_bytes(s) <= 0) return cudaErrorInvalidValue;
+    const MxPrepared m = mx_tc_prepared_parts(s, out);
+    // the scale atoms of GEMM 2 follow GEMM 1's after its 256-byte padding:
+    // two launches, one per GEMM, each with its own word range
+    const int64_t n_gu = mx_tc_tiled_gu_bytes(s) / 4, n_dn = mx_tc_tiled_dn_bytes(s) / 4;
+    mx_tc_tile_scales_kernel<<<grid_of(n_gu, num_sms), 256, 0, st>>>(
+        gu_s, dn_s, reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(m.tiled)), s.E, s.H, s.I,
+        n_gu, n_gu);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mx_tc_tile_scales_kernel<<<grid_of(n_dn, num_sms), 256, 0, st>>>(
+        gu_s, dn_s, reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(m.tiled_dn)), s.E, s.H, s.I,
+        0, n_dn);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (m.gu_codes) {
+        const int64_t rows = static_cast<int64_t>(s.E) * 2 * s.I;
+        const int Kp = static_cast<int>(round128(s.H));
+        mx_tc_pad_codes_kernel<<<grid_of(rows * (Kp / 32), num_sms), 256, 0, st>>>(
+            reinterpret_cast<const uint4*>(gu_q), reinterpret_cast<uint4*>(const_cast<uint8_t*>(m.gu_codes)),
+            rows, s.H, Kp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (m.dn_codes) {
+        const int64_t rows = static_cast<int64_t>(s.E) * s.H;
+        const int Kp = static_cast<int>(round128(s.I));
+        mx_tc_pad_codes_kernel<<<grid_of(rows * (Kp / 32), num_sms), 256, 0, st>>>(
+            reinterpret_cast<const uint4*>(dn_q), reinterpret_cast<uint4*>(const_cast<uint8_t*>(m.dn_codes)),
+            rows, s.I, Kp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// The tensor-core path takes H and I multiples of 64 with the prepared
+// weights, of 128 with the raw ones (whole 4-byte scale words per row).
+bool mx_tc_supported(const moe_shape& s, const void* gu_q, const void* dn_q, bool prepared) {
+    const bool shape_ok = prepared ? (s.H % 64 == 0 && s.I % 64 == 0)
+                                : (s.H % 128 == 0 && s.I % 128 == 0);
+    return shape_ok && s.T >= 1 && s.T <= 64 &&
            (reinterpret_cast<uintptr_t>(gu_q) & 31u) == 0 &&
            (reinterpret_cast<uintptr_t>(dn_q) & 31u) == 0;
 }
 
-template <int KIND, int CH, int KGS, int CPS>
+template <int KIND, int CH, int KGS, int CPS, bool TILED>
 static cudaError_t launch_tc(const CUtensorMap& mw, const CUtensorMap& ma, const MxTcParams& p,
                              int num_sms, cudaStream_t st) {
     using G = TcGeo<CH, KGS, CPS>;
-    auto kern = decode_mx_tc_kernel<KIND, CH, KGS, CPS>;
+    auto kern = decode_mx_tc_kernel<KIND, CH, KGS, CPS, TILED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          G::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(CPS * num_sms), dim3(mxtc::THREADS), G::SMEM_BYTES, st, mw, ma, p);
 }
 
-template <int CH, int KGS, int CPS>
+template <int CH, int KGS, int CPS, bool TILED>
 static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offsets,
                           const int32_t* perm, const float* topk_w, const uint8_t* gu_q,
                           const uint8_t* gu_s, const uint8_t* dn_q, const uint8_t* dn_s,
-                          uint8_t* xq, uint8_t* xsf, uint8_t* hq, uint8_t* hsf, float* part,
-                          int32_t* ctl, void* y_slots, int32_t* err_flag, int num_sms,
-                          cudaStream_t st) {
+                          const void* prepared, uint8_t* xq, uint8_t* xsf, uint8_t* hq,
+                          uint8_t* hsf, float* part, int32_t* ctl, void* y_slots,
+                          int32_t* err_flag, int num_sms, cudaStream_t st) {
     const int S = static_cast<int>(s.T * s.k);
     const int SP = static_cast<int>(mx_tc_plane_rows(S));
+    const MxPrepared m = TILED ? mx_tc_prepared_parts(s, prepared)
+                               : MxPrepared{nullptr, nullptr, nullptr, nullptr};
+    // codes: the padded copies where a row is not whole K-groups
+    const uint8_t* gu_codes = m.gu_codes ? m.gu_codes : gu_q;
+    const uint8_t* dn_codes = m.dn_codes ? m.dn_codes : dn_q;
+    const int64_t Kg = m.gu_codes ? round128(s.H) : s.H, Kd = m.dn_codes ? round128(s.I) : s.I;
     CUtensorMap map_gu, map_dn, map_x, map_h;
     // GEMM 1 rows: gate row i of expert e at e*2I + i, up at e*2I + I + i
     // GEMM 2 rows: row n of expert e at e*H + n, blocks of 64
-    if (!make_map_e2m1(&map_gu, gu_q, s.E, 2 * static_cast<int64_t>(s.I), s.H, s.I, 2, s.I, KGS) ||
-        !make_map_e2m1(&map_dn, dn_q, s.E, s.H, s.I, mxtc::HALF_ROWS, s.H / mxtc::HALF_ROWS,
-                       mxtc::HALF_ROWS, KGS) ||
-        !make_map_e4m3(&map_x, xq, SP, s.H, CH, KGS) || !make_map_e4m3(&map_h, hq, SP, s.I, CH, KGS))
+    if (!make_map_e2m1(&map_gu, gu_codes, s.E, 2 * static_cast<int64_t>(s.I), Kg, s.I, 2, s.I) ||
+        !make_map_e2m1(&map_dn, dn_codes, s.E, s.H, Kd, mxtc::HALF_ROWS, s.H / mxtc::HALF_ROWS,
+                       mxtc::HALF_ROWS) ||
+        !make_map_e4m3(&map_x, xq, SP, s.H, CH) || !make_map_e4m3(&map_h, hq, SP, s.I, CH))
         return cudaErrorInvalidValue;
+    const int sf_x = mx_tc_sf_stride(s.H), sf_h = mx_tc_sf_stride(s.I);
 
     constexpr int WPB = mxtc::PREP_THREADS / 32;
-    cudaError_t e = launch_pdl(mx_tc_prep_x_kernel, dim3((s.H / 32 + WPB - 1) / WPB, S),
+    cudaError_t e = launch_pdl(mx_tc_prep_x_kernel, dim3((sf_x + WPB - 1) / WPB, S),
                                dim3(mxtc::PREP_THREADS), 0, st,
-                               static_cast<const __nv_bfloat16*>(x), perm, s.k, s.H, SP, xq, xsf);
+                               static_cast<const __nv_bfloat16*>(x), perm, s.k, s.H, SP, sf_x, xq,
+                               xsf);
     if (e != cudaSuccess) return e;
 
     MxTcParams p{};
@@ -715,53 +912,75 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
     p.timeout_ns = 4000000000ull;
     // GEMM 1: gate_up, K = H, 64 gate + 64 up rows per tile
     p.w_scales = gu_s;
+    p.w_tiled = m.tiled;
     p.act_sf = xsf;
+    p.sf_stride = sf_x;
     p.K = s.H;
     p.wrows = 2 * static_cast<int64_t>(s.I);
     p.n_out = 2 * s.I;
     p.mtiles = s.I / mxtc::HALF_ROWS;
-    e = launch_tc<0, CH, KGS, CPS>(map_gu, map_x, p, num_sms, st);
+    e = launch_tc<0, CH, KGS, CPS, TILED>(map_gu, map_x, p, num_sms, st);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(mx_tc_swiglu_kernel, dim3((s.I / 32 + WPB - 1) / WPB, S),
-                   dim3(mxtc::PREP_THREADS), 0, st, part, ctl, S, s.I, SP, hq, hsf);
+    e = launch_pdl(mx_tc_swiglu_kernel, dim3((sf_h + WPB - 1) / WPB, S),
+                   dim3(mxtc::PREP_THREADS), 0, st, part, ctl, S, s.I, SP, sf_h, hq, hsf);
     if (e != cudaSuccess) return e;
-    // GEMM 2: down, K = I, 128 rows per tile
+    // GEMM 2: down, K = I, 128 rows per tile (the last one partial when H % 128 != 0)
     p.w_scales = dn_s;
+    p.w_tiled = m.tiled_dn;
     p.act_sf = hsf;
+    p.sf_stride = sf_h;
     p.K = s.I;
     p.wrows = s.H;
     p.n_out = s.H;
-    p.mtiles = s.H / 128;
-    e = launch_tc<1, CH, KGS, CPS>(map_dn, map_h, p, num_sms, st);
+    p.mtiles = (s.H + 127) / 128;
+    e = launch_tc<1, CH, KGS, CPS, TILED>(map_dn, map_h, p, num_sms, st);
     if (e != cudaSuccess) return e;
     return launch_pdl(mx_tc_down_out_kernel, dim3((s.H + 255) / 256, S), dim3(256), 0, st, part,
                       ctl, perm, topk_w, s.routed_scale, S, s.H,
                       static_cast<__nv_bfloat16*>(y_slots));
 }
 
-// moe_forward_mxfp4 on the block-scaled tensor cores (mx_tc_supported):
-// chunks of 8 rows per expert for batches of up to 8 tokens, else 16.  An
-// expert with more rows than a chunk streams its weights once per chunk (at
-// T = 64 over 16 experts a few do; chunks of 32 rows, which avoid that but
-// fit only two CTAs per SM with a single accumulator, measured 8 % slower).  Several CTAs per SM: each tcgen05 instruction costs its issuing
-// thread a roughly fixed time, so more issuing threads per SM move more
-// bytes (MxTcCfg: CTAs per SM and K-groups per stage by chunk size).
+template <bool TILED>
+static cudaError_t run_tc_t(const moe_shape& s, const void* x, const int32_t* offsets,
+                            const int32_t* perm, const float* topk_w, const uint8_t* gu_q,
+                            const uint8_t* gu_s, const uint8_t* dn_q, const uint8_t* dn_s,
+                            const void* prepared, uint8_t* xq, uint8_t* xsf, uint8_t* hq,
+                            uint8_t* hsf, float* part, int32_t* ctl, void* y_slots,
+                            int32_t* err_flag, int num_sms, cudaStream_t st) {
+    if (s.T <= 8)
+        return run_tc<8, MxTcCfg<8>::KGS, MxTcCfg<8>::CPS, TILED>(
+            s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, prepared, xq, xsf, hq, hsf, part,
+            ctl, y_slots, err_flag, num_sms, st);
+    return run_tc<16, MxTcCfg<16>::KGS, MxTcCfg<16>::CPS, TILED>(
+        s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, prepared, xq, xsf, hq, hsf, part,
+        ctl, y_slots, err_flag, num_sms, st);
+}
+
+// moe_forward_mxfp4 on the block-scaled tensor cores (mx_tc_supported), with
+// the raw weights (prepared == NULL) or the prepared ones: chunks of 8 rows
+// per expert for batches of up to 8 tokens, else 16.  An expert with more
+// rows than a chunk streams its weights once per chunk (at T = 64 over 16
+// experts a few do; chunks of 32 rows, which avoid that but fit only two CTAs
+// per SM with a single accumulator, measured 8 % slower).  Several CTAs per
+// SM: each tcgen05 instruction costs its issuing thread a roughly fixed time,
+// so more issuing threads per SM move more bytes (MxTcCfg: CTAs per SM and
+// K-groups per stage by chunk size).
 cudaError_t launch_ffn_decode_mxfp4_tc(const moe_shape& s, const void* x, const int32_t* offsets,
                                        const int32_t* perm, const float* topk_w,
                                        const uint8_t* gu_q, const uint8_t* gu_s,
-                                       const uint8_t* dn_q, const uint8_t* dn_s, uint8_t* xq,
-                                       uint8_t* xsf, uint8_t* hq, uint8_t* hsf, float* part,
-                                       int32_t* ctl, void* y_slots, int32_t* err_flag,
-                                       int num_sms, cudaStream_t st) {
-    if (!mx_tc_supported(s, gu_q, dn_q) || s.dtype != MOE_BF16 || s.n_shared != 0)
+                                       const uint8_t* dn_q, const uint8_t* dn_s,
+                                       const void* prepared, uint8_t* xq, uint8_t* xsf,
+                                       uint8_t* hq, uint8_t* hsf, float* part, int32_t* ctl,
+                                       void* y_slots, int32_t* err_flag, int num_sms,
+                                       cudaStream_t st) {
+    if (!mx_tc_supported(s, gu_q, dn_q, prepared != nullptr) || s.dtype != MOE_BF16 ||
+        s.n_shared != 0)
         return cudaErrorInvalidValue;
-    if (s.T <= 8)
-        return run_tc<8, MxTcCfg<8>::KGS, MxTcCfg<8>::CPS>(
-            s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, xq, xsf, hq, hsf, part, ctl,
-            y_slots, err_flag, num_sms, st);
-    return run_tc<16, MxTcCfg<16>::KGS, MxTcCfg<16>::CPS>(
-        s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, xq, xsf, hq, hsf, part, ctl, y_slots,
-        err_flag, num_sms, st);
+    if (prepared)
+        return run_tc_t<true>(s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, prepared, xq,
+                              xsf, hq, hsf, part, ctl, y_slots, err_flag, num_sms, st);
+    return run_tc_t<false>(s, x, offsets, perm, topk_w, gu_q, gu_s, dn_q, dn_s, prepared, xq,
+                           xsf, hq, hsf, part, ctl, y_slots, err_flag, num_sms, st);
 }
 
 }  // namespace moe

@@ -42,14 +42,17 @@ cudaError_t launch_ffn_decode_mxfp4(const moe_shape&, const void*, const int32_t
                                     int32_t*, void*, int32_t*, int, cudaStream_t);
 cudaError_t launch_combine(const moe_shape&, const void*, const int32_t*, void*, cudaStream_t);
 int mx_padded_cols(int K);
-bool mx_tc_supported(const moe_shape&, const void*, const void*);
+bool mx_tc_supported(const moe_shape&, const void*, const void*, bool);
+int64_t mx_tc_prepared_bytes(const moe_shape&);
+cudaError_t launch_mx_tc_prepare(const moe_shape&, const uint8_t*, const uint8_t*, const uint8_t*,
+                                 const uint8_t*, void*, int, cudaStream_t);
 int64_t mx_tc_plane_rows(int64_t slots);
 int64_t mx_tc_part_floats(int64_t slots, int H, int I);
 cudaError_t launch_ffn_decode_mxfp4_tc(const moe_shape&, const void*, const int32_t*,
                                        const int32_t*, const float*, const uint8_t*,
-                                       const uint8_t*, const uint8_t*, const uint8_t*, uint8_t*,
-                                       uint8_t*, uint8_t*, uint8_t*, float*, int32_t*, void*,
-                                       int32_t*, int, cudaStream_t);
+                                       const uint8_t*, const uint8_t*, const uint8_t*,
+                                       const void*, uint8_t*, uint8_t*, uint8_t*, uint8_t*,
+                                       float*, int32_t*, void*, int32_t*, int, cudaStream_t);
 cudaError_t launch_combine_experts(const moe_shape&, int, int, int, const void*, const int32_t*,
                                    const int32_t*, float*, int, cudaStream_t);
 cudaError_t launch_cast_f32(const moe_shape&, const float*, void*, int, cudaStream_t);
@@ -147,18 +150,19 @@ Workspace layout(const moe_shape& s) {
         off += align_up(static_cast<size_t>(Tk) * moe::mx_padded_cols(s.I) * 2);
         w.mx_hexp_off = off;
         off += align_up(static_cast<size_t>(Tk) * 4);
-        if (s.H % 128 == 0 && s.I % 128 == 0) {
+        if (s.H % 64 == 0 && s.I % 64 == 0) {
             // block-scaled tensor-core path: E4M3 hi/lo planes of x and h with
-            // their exponents, the split partials, and the split count
+            // their exponents (rows of 4 bytes per 128-column K-group), the
+            // split partials, and the split count
             const size_t SP = static_cast<size_t>(moe::mx_tc_plane_rows(Tk));
             w.mx_xq_off = off;
             off += align_up(2 * SP * s.H);
             w.mx_xsf_off = off;
-            off += align_up(2 * SP * (s.H / 32));
+            off += align_up(2 * SP * ((s.H + 127) / 128 * 4));
             w.mx_hq_off = off;
             off += align_up(2 * SP * s.I);
             w.mx_hsf_off = off;
-            off += align_up(2 * SP * (s.I / 32));
+            off += align_up(2 * SP * ((s.I + 127) / 128 * 4));
             w.mx_part_off = off;
             off += align_up(static_cast<size_t>(moe::mx_tc_part_floats(Tk, s.H, s.I)) * 4);
             w.mx_ctl_off = off;
@@ -648,9 +652,9 @@ moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x, const int32_
     if ((reinterpret_cast<uintptr_t>(gate_up_s) & 3u) || (reinterpret_cast<uintptr_t>(down_s) & 3u))
         return MOE_ERR_UNSUPPORTED;
     char* ws = static_cast<char*>(workspace);
-    if (moe::mx_tc_supported(s, gate_up_q, down_q))
+    if (moe::mx_tc_supported(s, gate_up_q, down_q, false))
         return cuda_status(moe::launch_ffn_decode_mxfp4_tc(
-            s, x, offsets, perm, topk_w, gate_up_q, gate_up_s, down_q, down_s,
+            s, x, offsets, perm, topk_w, gate_up_q, gate_up_s, down_q, down_s, nullptr,
             reinterpret_cast<uint8_t*>(ws + w.mx_xq_off), reinterpret_cast<uint8_t*>(ws + w.mx_xsf_off),
             reinterpret_cast<uint8_t*>(ws + w.mx_hq_off), reinterpret_cast<uint8_t*>(ws + w.mx_hsf_off),
             reinterpret_cast<float*>(ws + w.mx_part_off), reinterpret_cast<int32_t*>(ws + w.mx_ctl_off),
@@ -660,6 +664,60 @@ moe_status moe_forward_mxfp4(const moe_shape* shape, const void* x, const int32_
         ws + w.mx_x16_off, reinterpret_cast<int32_t*>(ws + w.mx_xexp_off), ws + w.mx_h16_off,
         reinterpret_cast<int32_t*>(ws + w.mx_hexp_off), y_slots, err_flag, num_sms(),
         static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_mxfp4_prepared_size(const moe_shape* shape, size_t* bytes) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = static_cast<size_t>(moe::mx_tc_prepared_bytes(*shape));
+    return MOE_OK;
+}
+
+moe_status moe_mxfp4_prepare(const moe_shape* shape, const uint8_t* gate_up_q,
+                             const uint8_t* gate_up_s, const uint8_t* down_q,
+                             const uint8_t* down_s, void* prepared, size_t prepared_bytes,
+                             void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    const size_t need = static_cast<size_t>(moe::mx_tc_prepared_bytes(*shape));
+    if (need == 0) return MOE_ERR_UNSUPPORTED;
+    if (!gate_up_q || !gate_up_s || !down_q || !down_s || !prepared) return MOE_ERR_INVALID_ARG;
+    if (prepared_bytes < need) return MOE_ERR_WORKSPACE;
+    if (!aligned16(prepared) || !aligned16(gate_up_q) || !aligned16(down_q))
+        return MOE_ERR_UNSUPPORTED;
+    return cuda_status(moe::launch_mx_tc_prepare(*shape, gate_up_q, gate_up_s, down_q, down_s,
+                                                 prepared, num_sms(),
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward_mxfp4_prepared(const moe_shape* shape, const void* x,
+                                      const int32_t* offsets, const int32_t* perm,
+                                      const float* topk_w, const uint8_t* gate_up_q,
+                                      const uint8_t* down_q, const void* prepared, void* y_slots,
+                                      int32_t* err_flag, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    const moe_shape& s = *shape;
+    if (s.T == 0) return MOE_OK;
+    if (s.dtype != MOE_BF16 || s.n_shared != 0 || s.T > 64 || s.H % 64 != 0 || s.I % 64 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (!x || !offsets || !perm || !topk_w || !gate_up_q || !down_q || !prepared || !y_slots)
+        return MOE_ERR_INVALID_ARG;
+    const Workspace w = layout(s);
+    if (!workspace || workspace_bytes < w.total) return MOE_ERR_WORKSPACE;
+    const void* ptrs[] = {x, gate_up_q, down_q, prepared, y_slots, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
+    if (!moe::mx_tc_supported(s, gate_up_q, down_q, true)) return MOE_ERR_UNSUPPORTED;
+    char* ws = static_cast<char*>(workspace);
+    return cuda_status(moe::launch_ffn_decode_mxfp4_tc(
+        s, x, offsets, perm, topk_w, gate_up_q, nullptr, down_q, nullptr, prepared,
+        reinterpret_cast<uint8_t*>(ws + w.mx_xq_off), reinterpret_cast<uint8_t*>(ws + w.mx_xsf_off),
+        reinterpret_cast<uint8_t*>(ws + w.mx_hq_off), reinterpret_cast<uint8_t*>(ws + w.mx_hsf_off),
+        reinterpret_cast<float*>(ws + w.mx_part_off), reinterpret_cast<int32_t*>(ws + w.mx_ctl_off),
+        y_slots, err_flag, num_sms(), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* inv, void* y,

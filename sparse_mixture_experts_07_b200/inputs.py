@@ -82,6 +82,9 @@ CONFIGS = {
     "phimoe_decode8": MoEConfig("phimoe_decode8", T=8, H=4096, I=6400, E=16, k=2),
     "phimoe_decode64": MoEConfig("phimoe_decode64", T=64, H=4096, I=6400, E=16, k=2),
     "gptoss": MoEConfig("gptoss", T=16384, H=2880, I=2880, E=32, k=4, zipf_s=1.0),
+    # decode batches of the same layer (gpt-oss stores its experts in mxfp4)
+    "gptoss_decode1": MoEConfig("gptoss_decode1", T=1, H=2880, I=2880, E=32, k=4, zipf_s=1.0),
+    "gptoss_decode8": MoEConfig("gptoss_decode8", T=8, H=2880, I=2880, E=32, k=4, zipf_s=1.0),
     "dsv3": MoEConfig("dsv3", T=32768, H=2048, I=1024, E=64, k=6, n_shared=2,
                       I_shared=1024, routed_scale=2.5, zipf_s=1.2),
     # the same layer with the DeepSeek-V3 routing the Instella page names

@@ -60,6 +60,10 @@ def load_library(path: str = LIB_PATH):
     lib.moe_permute.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_route_permute.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                       ctypes.c_size_t, P]
+    lib.moe_mxfp4_prepared_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
+    lib.moe_mxfp4_prepare.argtypes = [S, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.moe_forward_mxfp4_prepared.argtypes = [S, P, P, P, P, P, P, P, P, P, P,
+                                               ctypes.c_size_t, P]
     lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_combine.argtypes = [S, P, P, P, P]
     lib.moe_router_split_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
@@ -267,6 +271,40 @@ def forward_mxfp4(shape: Shape, x, offsets, perm, topk_w, mxfp4: dict, workspace
     return y_slots
 
 
+def mxfp4_prepare(shape: Shape, mxfp4: dict, stream=None):
+    """`mxfp4` prepared once for the tensor-core kernel (moe_mxfp4_prepare: the
+    scales in tensor-memory order, codes padded to whole 128-weight groups
+    where H or I needs it): a uint8 device tensor, or None when the shape
+    cannot take it (H or I not a multiple of 64)."""
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    _check(lib.moe_mxfp4_prepared_size(ctypes.byref(shape.c()), ctypes.byref(n)),
+           "moe_mxfp4_prepared_size")
+    if n.value == 0:
+        return None
+    prepared = torch.empty(n.value, dtype=torch.uint8, device=mxfp4["gate_up_s"].device)
+    _check(lib.moe_mxfp4_prepare(ctypes.byref(shape.c()), _ptr(mxfp4["gate_up_q"]),
+                                 _ptr(mxfp4["gate_up_s"]), _ptr(mxfp4["down_q"]),
+                                 _ptr(mxfp4["down_s"]), _ptr(prepared), n.value,
+                                 _stream(stream)), "moe_mxfp4_prepare")
+    return prepared
+
+
+def forward_mxfp4_prepared(shape: Shape, x, offsets, perm, topk_w, mxfp4: dict, prepared,
+                           workspace, err_flag, y_slots=None, stream=None):
+    """moe_forward_mxfp4 on the tensor cores with the prepared weights (H and I
+    multiples of 64): `mxfp4` supplies the raw gate_up_q and down_q."""
+    lib = load_library()
+    if y_slots is None:
+        y_slots = torch.empty(shape.slot_rows, shape.H, dtype=shape.torch_dtype, device=x.device)
+    _check(lib.moe_forward_mxfp4_prepared(ctypes.byref(shape.c()), _ptr(x), _ptr(offsets),
+                                          _ptr(perm), _ptr(topk_w), _ptr(mxfp4["gate_up_q"]),
+                                          _ptr(mxfp4["down_q"]), _ptr(prepared), _ptr(y_slots),
+                                          _ptr(err_flag), _ptr(workspace), workspace.numel(),
+                                          _stream(stream)), "moe_forward_mxfp4_prepared")
+    return y_slots
+
+
 def forward_experts(shape: Shape, e_begin: int, e_end: int, x, offsets, perm, topk_w,
                     gate_up_local, down_local, sh_gate_up, sh_down, workspace, err_flag,
                     y_slots, stream=None):
@@ -404,6 +442,12 @@ class MoELayer:
         self.w_split = router_split(shape, w_router)
         self.gate_up, self.down = gate_up, down
         self.sh_gate_up, self.sh_down = sh_gate_up, sh_down
+        # MXFP4 weights prepared once for the tensor-core kernel where it
+        # takes the shape (decode batches, H and I multiples of 64)
+        self.mx_prepared = None
+        if (mxfp4 is not None and 1 <= shape.T <= 64 and shape.n_shared == 0
+                and shape.dtype == MOE_BF16):
+            self.mx_prepared = mxfp4_prepare(shape, mxfp4)
         dev = (gate_up if mxfp4 is None else mxfp4["gate_up_q"]).device
         self.workspace = alloc_workspace(shape, dev)
         self.err_flag = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -435,7 +479,11 @@ class MoELayer:
             idx, w, _, counts, offsets, perm, inv = route_permute(
                 s, x, self.w_router, self.router_bias, self.workspace, self.err_flag, out=b,
                 stream=stream, w_split=self.w_split)
-        if self.mxfp4 is not None:
+        if self.mx_prepared is not None:
+            forward_mxfp4_prepared(s, x, offsets, perm, w, self.mxfp4, self.mx_prepared,
+                                   self.workspace, self.err_flag, y_slots=b["y_slots"],
+                                   stream=stream)
+        elif self.mxfp4 is not None:
             forward_mxfp4(s, x, offsets, perm, w, self.mxfp4, self.workspace, self.err_flag,
                           y_slots=b["y_slots"], stream=stream)
         else:

@@ -235,3 +235,54 @@ def test_noaux_rejects_bad_group_arguments(lib, n_group, topk_group):
     assert f(ctypes.byref(s), n_group, topk_group, p, p, None, None, p, p, p, None, None) == 1
     # valid groups, but the logits buffer the selection reads is required
     assert f(ctypes.byref(s), 4, 2, p, p, None, None, None, p, p, None, None) == 1
+
+
+def _prepared_size(lib, s):
+    n = ctypes.c_size_t(0)
+    rc = lib.moe_mxfp4_prepared_size(ctypes.byref(s), ctypes.byref(n))
+    return rc, n.value
+
+
+def _prepared_bytes(H, I, E):
+    """Scale atoms of both GEMMs, then codes padded to 128-weight rows where
+    H or I needs it; each part rounded up to 256 bytes."""
+    def a256(v):
+        return (v + 255) // 256 * 256
+    def c128(v):
+        return -(-v // 128)
+    parts = [512 * E * (I // 64) * c128(H), 512 * E * c128(H) * c128(I),
+             E * 2 * I * c128(H) * 64 if H % 128 else 0, E * H * c128(I) * 64 if I % 128 else 0]
+    return sum(a256(p) for p in parts)
+
+
+@pytest.mark.parametrize("H,I,E", [(4096, 6400, 16), (2880, 2880, 32), (320, 192, 3),
+                                   (288, 128, 8), (256, 96, 8)])
+def test_mxfp4_prepared_size(lib, H, I, E):
+    want = _prepared_bytes(H, I, E) if H % 64 == 0 and I % 64 == 0 else 0
+    assert _prepared_size(lib, _shape(H=H, I=I, E=E, k=2, T=8)) == (0, want)
+    if (H, I, E) == (4096, 6400, 16):
+        assert want == 512 * 16 * (100 * 32 + 32 * 50)       # no padded codes
+
+
+def test_mxfp4_prepared_argument_checks(lib):
+    s = _shape(H=320, I=192, E=4, k=2, T=8)
+    _, need = _prepared_size(lib, s)
+    ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 8)
+    assert lib.moe_mxfp4_prepare(ctypes.byref(s), None, ok, ok, ok, ok, need, None) == 1
+    assert lib.moe_mxfp4_prepare(ctypes.byref(s), ok, ok, ok, ok, ok, need - 1, None) == 3
+    assert lib.moe_mxfp4_prepare(ctypes.byref(s), ok, ok, ok, ok, bad, need, None) == 2
+    odd = _shape(H=288, I=192, E=4, k=2, T=8)
+    assert lib.moe_mxfp4_prepare(ctypes.byref(odd), ok, ok, ok, ok, ok, 1 << 30, None) == 2
+    _, ws = _ws(lib, s)
+    # x, offsets, perm, topk_w, gate_up_q, down_q, prepared, y_slots
+    args = [ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ws, None]
+    for i in range(8):
+        a = list(args)
+        a[i] = None
+        assert lib.moe_forward_mxfp4_prepared(ctypes.byref(s), *a) == 1, i
+    a = list(args)
+    a[9] = None
+    assert lib.moe_forward_mxfp4_prepared(ctypes.byref(s), *a) == 3
+    assert lib.moe_forward_mxfp4_prepared(ctypes.byref(odd), *args) == 2
+    long_batch = _shape(H=320, I=192, E=4, k=2, T=65)
+    assert lib.moe_forward_mxfp4_prepared(ctypes.byref(long_batch), *args) == 2

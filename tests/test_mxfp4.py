@@ -31,7 +31,16 @@ SMALL = [
     MoEConfig("mx_tc_T64_two_chunks", T=64, H=256, I=256, E=4, k=2, zipf_s=1.2),
     MoEConfig("mx_tc_splits", T=1, H=2176, I=1152, E=8, k=2),
     MoEConfig("mx_tc_T33_splits", T=33, H=1024, I=512, E=32, k=2, zipf_s=1.0),
+    # H and I multiples of 64 but not of 128 (gpt-oss's 2880 is one): the
+    # tensor-core kernel on prepared weights (padded rows), a partial last
+    # K-group of the activations and, in GEMM 2, a partial last 128-row tile
+    MoEConfig("mx_tiled_gptoss_like_T1", T=1, H=320, I=320, E=32, k=4, zipf_s=1.0),
+    MoEConfig("mx_tiled_T7", T=7, H=576, I=192, E=16, k=4, routed_scale=2.5),
+    MoEConfig("mx_tiled_T33", T=33, H=448, I=320, E=32, k=4, zipf_s=1.0),
+    MoEConfig("mx_tiled_T64_splits", T=64, H=2880, I=320, E=8, k=2),
 ]
+# (H, I multiples of 128) run on both weight forms: raw and prepared agree bit for bit
+RAW_AND_TILED = [c for c in SMALL if c.H % 128 == 0 and c.I % 128 == 0]
 
 
 def _run(cfg, inp, mw):
@@ -67,6 +76,91 @@ def test_mxfp4_decode_small(cuda_ok, cfg):
     inp = make_inputs(cfg)
     mw = make_mxfp4_weights(cfg)
     layer, y = _run(cfg, inp, mw)
+    _check(cfg, inp, mw, layer, y)
+
+
+@pytest.mark.parametrize("cfg", RAW_AND_TILED, ids=lambda c: c.name)
+def test_mxfp4_raw_and_prepared_agree(cuda_ok, cfg):
+    """moe_forward_mxfp4 (raw [rows, K/32] scales, per-row copies) and
+    moe_forward_mxfp4_prepared (the same scales re-laid out once) run the same
+    arithmetic: outputs equal bit for bit; the raw path matches the oracle."""
+    import sparse_mixture_experts_07_b200 as moe
+    inp = make_inputs(cfg)
+    mw = make_mxfp4_weights(cfg)
+    layer, y_prep = _run(cfg, inp, mw)
+    assert layer.mx_prepared is not None
+    b = layer.last
+    y_raw = moe.forward_mxfp4(layer.shape, to_device(inp)["x"], b["offsets"], b["perm"],
+                              b["topk_w"], layer.mxfp4, layer.workspace, layer.err_flag)
+    y_raw = moe.combine(layer.shape, y_raw, b["inv"]).cpu()
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    assert torch.equal(y_raw, y_prep)
+    _check(cfg, inp, mw, layer, y_raw)
+
+
+def _a256(v):
+    return (v + 255) // 256 * 256
+
+
+def test_mxfp4_prepared_layout(cuda_ok):
+    """The prepared array holds, for every (expert, tile, K-group, word, byte),
+    the raw scale of the row and block its layout names (127 past the rows
+    and blocks), then the codes of both weights with rows padded by zero
+    bytes to whole 128-weight groups (H = 320 and I = 192 both need it)."""
+    import sparse_mixture_experts_07_b200 as moe
+    cfg = MoEConfig("mx_prepare_layout", T=1, H=320, I=192, E=3, k=1)
+    mw = make_mxfp4_weights(cfg)
+    shape = moe.Shape.from_config(cfg)
+    prepared = moe.mxfp4_prepare(shape, {key: v.cuda() for key, v in mw.items()})
+    torch.cuda.synchronize()
+    got = prepared.cpu().numpy()
+    E, H, I = cfg.E, cfg.H, cfg.I
+    parts = []
+    for gemm in ("gu", "dn"):
+        K = H if gemm == "gu" else I
+        raw = (mw["gate_up_s"] if gemm == "gu" else mw["down_s"]).numpy()
+        mtiles = I // 64 if gemm == "gu" else -(-H // 128)
+        atoms = []
+        for e in range(E):
+            for mt in range(mtiles):
+                for kg in range(-(-K // 128)):
+                    atom = np.full(512, 127, dtype=np.uint8)
+                    for w in range(128):
+                        m = (w >> 2) + 32 * (w & 3)
+                        if gemm == "gu":
+                            row = mt * 64 + m if m < 64 else I + mt * 64 + (m - 64)
+                        else:
+                            row = mt * 128 + m
+                            if row >= H:
+                                continue
+                        for kb in range(4):
+                            blk = 4 * kg + kb
+                            if blk < K // 32:
+                                atom[4 * w + kb] = raw[e, row, blk]
+                    atoms.append(atom)
+        parts.append(np.concatenate(atoms))
+    for q, K in ((mw["gate_up_q"].numpy(), H), (mw["down_q"].numpy(), I)):
+        Kp = -(-K // 128) * 128
+        padded = np.zeros(q.shape[:-1] + (Kp // 2,), dtype=np.uint8)
+        padded[..., :K // 2] = q
+        parts.append(padded.reshape(-1))
+    off = 0
+    for part in parts:
+        assert np.array_equal(got[off:off + part.size], part)
+        off = _a256(off + part.size)
+    assert off == got.size
+
+
+@pytest.mark.parametrize("name", ["gptoss_decode1", "gptoss_decode8"])
+def test_mxfp4_decode_gptoss_full_size(cuda_ok, name):
+    """gpt-oss-shaped layer (H = I = 2880, 32 experts, k = 4): the prepared
+    tensor-core path at full size against the oracle."""
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg)
+    mw = make_mxfp4_weights(cfg)
+    layer, y = _run(cfg, inp, mw)
+    assert layer.mx_prepared is not None
     _check(cfg, inp, mw, layer, y)
 
 
