@@ -274,7 +274,8 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const int3
  * T*k routed rows).  Supported: bf16 x, 1 <= T <= 64, no shared experts, H
  * and I multiples of 32, the scale arrays 4-byte aligned; otherwise
  * MOE_ERR_UNSUPPORTED.  Two kernels, chosen by shape:
- *   - H and I multiples of 128 and the code arrays 32-byte aligned: the
+ *   - H and I multiples of 128 and the code arrays 32-byte aligned (64 with
+ *     moe_forward_mxfp4_prepared below): the
  *     block-scaled tensor-core MMA (E2M1 weights x E4M3 activations, E8M0
  *     scales on both).  Each bf16 activation (x, then h rounded to bf16) is
  *     split per block of 32 into two E4M3 parts under E8M0 exponents, which
