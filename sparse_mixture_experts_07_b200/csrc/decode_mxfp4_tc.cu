@@ -9,9 +9,15 @@
 // as in the CUDA-core kernel: q [rows, K/2] bytes (element 2j in the low
 // nibble of byte j), s [rows, K/32] bytes.
 //
-// This path needs K % 128 == 0 for both GEMMs (H and I), and so covers
-// PhiMoE-, Mixtral- and DeepSeek-shaped layers; others take the CUDA-core
-// kernel.  Per MMA (M = 128, N = 2 CH, K = 32):
+// This path takes H and I multiples of 64 on weights prepared once
+// (mx_tc_prepare: the scales in tensor-memory order; codes padded to whole
+// 128-weight groups where H or I is not a multiple of 128, the 4-bit
+// unpacking tensor maps taking only those), which covers gpt-oss's 2880 as
+// well as PhiMoE-, Mixtral- and DeepSeek-shaped layers, and multiples of 128
+// on the raw arrays; other shapes take the CUDA-core kernel.  The
+// activations' last K-group is zero past K (tensor-map fill), so whatever
+// padded weight codes meet there contribute nothing.  Per MMA (M = 128,
+// N = 2 CH, K = 32):
 //   A  128 weight rows.  TMA reads the packed codes with the 16U4_ALIGN16B
 //      element type, which spreads every 16 codes (8 bytes in memory) over
 //      16 bytes of shared memory: the layout this MMA kind reads 4-bit
@@ -42,11 +48,13 @@
 // Persistent CTAs of 192 threads, two or three per SM (MxTcCfg): a
 // tcgen05 instruction costs its issuing thread a roughly fixed time whatever
 // its size, so the SM moves more bytes with more issuing threads.  Stages of
-// one K-group, weights as a 5D tensor-map box (the tile's two 64-row halves).
+// one K-group, weights as a 4D tensor-map box (the tile's two 64-row halves).
 //   warp 0     producer: lane 0 issues the TMA boxes of a stage (the weight
-//              tile, the hi and lo activation rows); all 32 lanes copy the
-//              stage's scale words with 4-byte cp.async and report them on
-//              the stage barrier with cp.async.mbarrier.arrive;
+//              tile, the hi and lo activation rows) and, on prepared
+//              weights, the bulk copy of the stage's weight-scale atom; all
+//              32 lanes copy the activation scale words (and, on raw
+//              weights, the weight scale words) with 4-byte cp.async and
+//              report them on the stage barrier with cp.async.mbarrier.arrive;
 //   warp 1     allocates tensor memory; one thread copies the stage's scale
 //              factors to tensor memory and issues its four MMAs;
 //   warps 2-5  epilogue: tcgen05.ld of their 32 lanes, hi + lo, fp32 partial
