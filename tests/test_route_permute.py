@@ -50,3 +50,44 @@ def test_route_permute_equals_the_two_calls(cfg):
     assert np.array_equal(fused[0].cpu().numpy(), o_idx)
     for got, want in zip(fused[3:], oracle.permute(o_idx, cfg.E)):
         assert np.array_equal(got.cpu().numpy(), want)
+
+
+def _sweep_cases(n=24, seed=11):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        E = int(rng.choice([4, 8, 16, 32, 64, 128, 256]))
+        k = int(rng.integers(1, min(E, 16) + 1))
+        T = int(rng.integers(1, 17))
+        H = int(rng.choice([8, 64, 200, 512, 1000, 2048]))
+        cases.append((i, T, H, E, k, bool(rng.integers(0, 2))))
+    return cases
+
+
+@pytest.mark.parametrize("case", _sweep_cases(), ids=lambda c: f"sweep{c[0]}_T{c[1]}_H{c[2]}_E{c[3]}_k{c[4]}")
+def test_route_permute_sweep_one_launch(case):
+    """Random decode shapes on the one-launch path (T <= 16): routing and plan
+    equal the two separate calls bit for bit (both run the same router, so
+    near-ties resolve the same way), and the plan's invariants hold."""
+    import sparse_mixture_experts_07_b200 as moe
+    _, T, H, E, k, with_bias = case
+    shape = moe.Shape(T=T, H=H, I=64, E=E, k=k)
+    g = torch.Generator().manual_seed(T * 1000 + E * 10 + k)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16).cuda()
+    wr = (torch.randn(E, H, generator=g) * 0.05).cuda()
+    bias = (torch.randn(E, generator=g) * 0.5).cuda() if with_bias else None
+    ws = moe.alloc_workspace(shape)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fused = moe.route_permute(shape, x, wr, bias, ws, err, logits=True)
+    idx, w, lg = moe.route(shape, x, wr, bias, logits=True, err_flag=err)
+    plan = moe.permute(shape, idx, ws, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for a, b in zip(fused, (idx, w, lg) + tuple(plan)):
+        assert torch.equal(a, b)
+    counts, offsets, perm, inv = (t.cpu().numpy() for t in fused[3:])
+    sel = fused[0].cpu().numpy().reshape(-1)
+    assert counts.sum() == T * k and offsets[0] == 0 and np.array_equal(np.diff(offsets), counts)
+    assert np.array_equal(inv[perm], np.arange(T * k))
+    keys = sel[perm].astype(np.int64) * (T * k) + perm
+    assert np.all(np.diff(keys) > 0)
