@@ -79,6 +79,7 @@ constexpr int SPLIT_SLOTS = 128;           // splits x slots <= max(SPLIT_SLOTS,
 constexpr int MIN_KG_PER_SPLIT = 8;
 constexpr int PREP_THREADS = 256;          // 8 warps, one 32-block each
 constexpr int SMEM_BUDGET = 220 * 1024;
+constexpr int SF_PAD_ROWS = 16;            // a chunk's copy of CH rows stays in the block
 }  // namespace mxtc
 
 // CTAs per SM (CPS) and K-groups per stage (KGS) by chunk size CH: as many
@@ -127,8 +128,10 @@ struct MxTcParams {
     const int32_t* offsets;     // [E+1]
     const uint8_t* w_scales;    // [E * wrows, K/32] E8M0 of the weights (K a multiple of 128)
     const uint8_t* w_tiled;     // or: the weights' E8M0 in tensor-memory order (mx_tc_prepare)
-    const uint8_t* act_sf;      // [2 * SP, sf_stride] E8M0 of the activation planes (hi, then lo)
-    int sf_stride;              // bytes per activation scale row: 4 per K-group
+    const uint8_t* act_sf;      // E8M0 of the activation planes, per K-group kg a block of
+                                // sf_rows 16-byte rows (hi rows, lo rows at SP, padding):
+                                // row r, K-block kb at (kg * sf_rows + r) * 16 + kb
+    int sf_rows;                // 2 SP + SF_PAD_ROWS
     float* part;                // [splits][S][n_out] fp32 partial sums
     int32_t* ctl;               // ctl[0]: splits used (written by CTA 0)
     int32_t* err_flag;
@@ -301,7 +304,8 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int i = 0; i < G::STAGES; ++i) {
-            mbar_init(&full[i], 1 + 32);    // expect_tx arrival + one cp.async arrival per lane
+            // expect_tx arrival (+ one cp.async arrival per lane for raw weight scales)
+            mbar_init(&full[i], TILED ? 1 : 1 + 32);
             mbar_init(&empty[i], 1);        // tcgen05.commit
         }
         for (int b = 0; b < 2; ++b) {
@@ -391,35 +395,30 @@ __global__ void __launch_bounds__(mxtc::THREADS, CPS) decode_mx_tc_kernel(
                 if (lane == 0) {
                     // whole boxes always (codes past K and weight rows past the
                     // expert's are zero filled)
-                    mbar_arrive_expect_tx(&full[slot], G::TX + (TILED ? SF_ATOM : 0));
+                    mbar_arrive_expect_tx(&full[slot],
+                                          G::TX + 2 * CH * 16 + (TILED ? SF_ATOM : 0));
                     if (KIND == 0)
                         tma_load_4d(sa, &map_w, &full[slot], kg * KG, mt * HALF_ROWS, 0, grp);
                     else
                         tma_load_4d(sa, &map_w, &full[slot], kg * KG, 0, 2 * mt, grp);
                     tma_load_3d(sb, &map_act, &full[slot], kg * KG, brow0, 0);
                     if (TILED) bulk_load(sfa, tsrc + static_cast<int64_t>(kg) * SF_ATOM, SF_ATOM, &full[slot]);
+                    // the chunk's activation scales: CH hi rows then CH lo rows,
+                    // 16 bytes each, row n of the atom at byte 16 n (rows past
+                    // the slots feed columns nothing reads)
+                    const uint8_t* sfk = p.act_sf + static_cast<int64_t>(kg) * p.sf_rows * 16;
+                    bulk_load(sfb, sfk + static_cast<int64_t>(brow0) * 16, CH * 16, &full[slot]);
+                    bulk_load(sfb + CH * 16, sfk + static_cast<int64_t>(p.SP + brow0) * 16, CH * 16,
+                              &full[slot]);
                 }
-                for (int c = 0; c < nk; ++c) {
-                    if (!TILED) {
+                if (!TILED) {
+                    for (int c = 0; c < nk; ++c) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
                             cp_async4_tc(sfa + c * SF_ATOM + 4 * (32 * j + lane), wsrc[j] + 4 * (kg + c), 4u);
                     }
-#pragma unroll
-                    for (int j = 0; j < (G::N + 31) / 32; ++j) {
-                        const int n = lane + 32 * j;
-                        if (n < G::N) {
-                            const int plane = n / CH;
-                            const int srow = brow0 + (n - plane * CH);
-                            const bool in = srow < p.S;          // rows past the slots: zeros
-                            const uint8_t* src = p.act_sf +
-                                (static_cast<int64_t>(plane) * p.SP + (in ? srow : 0)) * p.sf_stride +
-                                4 * (kg + c);
-                            cp_async4_tc(sfb + c * SF_ATOM + 16 * lane + 4 * j, src, in ? 4u : 0u);
-                        }
-                    }
+                    cp_async_arrive_noinc_tc(&full[slot]);
                 }
-                cp_async_arrive_noinc_tc(&full[slot]);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
@@ -567,11 +566,16 @@ __device__ __forceinline__ float warp_max_abs(float v) {
     return m;
 }
 
+// Byte of activation scale row r, 32-block blk, in the layout the kernel
+// copies per K-group (MxTcParams::act_sf).
+__device__ __forceinline__ int64_t act_sf_byte(int64_t r, int blk, int sf_rows) {
+    return ((static_cast<int64_t>(blk >> 2) * sf_rows) + r) * 16 + (blk & 3);
+}
+
 // One warp per (slot row, 32-block): writes the value's hi byte to plane 0
-// (row r) and lo byte to plane 1 (row SP + r), and the exponents likewise
-// (scale rows of sf_stride bytes).
+// (row r) and lo byte to plane 1 (row SP + r), and the exponents likewise.
 __device__ __forceinline__ void store_e4m3_pair(float v, int64_t r, int blk, int K, int SP,
-                                                int sf_stride, uint8_t* q, uint8_t* sf) {
+                                                int sf_rows, uint8_t* q, uint8_t* sf) {
     const int lane = threadIdx.x & 31;
     const float bmax = warp_max_abs(v);
     uint8_t hi, lo;
@@ -580,20 +584,20 @@ __device__ __forceinline__ void store_e4m3_pair(float v, int64_t r, int blk, int
     q[r * K + blk * 32 + lane] = hi;
     q[(SP + r) * K + blk * 32 + lane] = lo;
     if (lane == 0) {
-        sf[r * sf_stride + blk] = static_cast<uint8_t>(eh + 127);
-        sf[(SP + r) * sf_stride + blk] = static_cast<uint8_t>(el + 127);
+        sf[act_sf_byte(r, blk, sf_rows)] = static_cast<uint8_t>(eh + 127);
+        sf[act_sf_byte(SP + r, blk, sf_rows)] = static_cast<uint8_t>(el + 127);
     }
 }
 
 // Scale bytes of the blocks past K that fill the last K-group (K % 128 != 0):
 // 2^0, a finite factor for codes the tensor map reads as zero.  True when
-// `blk` is such a block (written) or past the row (nothing to do).
-__device__ __forceinline__ bool pad_scale_block(int64_t r, int blk, int K, int SP, int sf_stride,
+// `blk` is such a block (written) or past the last K-group (nothing to do).
+__device__ __forceinline__ bool pad_scale_block(int64_t r, int blk, int K, int SP, int sf_rows,
                                                 uint8_t* sf) {
     if (blk < K / 32) return false;
-    if (blk < sf_stride && (threadIdx.x & 31) == 0) {
-        sf[r * sf_stride + blk] = 127;
-        sf[(SP + r) * sf_stride + blk] = 127;
+    if (blk < (K + mxtc::KG - 1) / mxtc::KG * 4 && (threadIdx.x & 31) == 0) {
+        sf[act_sf_byte(r, blk, sf_rows)] = 127;
+        sf[act_sf_byte(SP + r, blk, sf_rows)] = 127;
     }
     return true;
 }
@@ -601,27 +605,27 @@ __device__ __forceinline__ bool pad_scale_block(int64_t r, int blk, int K, int S
 // GEMM 1 operand B: x[perm[r] / k] of every sorted slot row r.
 __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_prep_x_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int k, int K, int SP,
-    int sf_stride, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    int sf_rows, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
     pdl_launch_dependents();
     pdl_wait();
     const int r = blockIdx.y;
     const int blk = blockIdx.x * (mxtc::PREP_THREADS / 32) + (threadIdx.x >> 5);
-    if (pad_scale_block(r, blk, K, SP, sf_stride, sf)) return;
+    if (pad_scale_block(r, blk, K, SP, sf_rows, sf)) return;
     const int64_t tok = perm[r] / k;
     const float v = __bfloat162float(x[tok * K + blk * 32 + (threadIdx.x & 31)]);
-    store_e4m3_pair(v, r, blk, K, SP, sf_stride, q, sf);
+    store_e4m3_pair(v, r, blk, K, SP, sf_rows, q, sf);
 }
 
 // GEMM 1 epilogue: gate and up summed over the splits in order, h =
 // SiLU(gate) * up rounded to bf16, then quantised as GEMM 2's operand B.
 __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_swiglu_kernel(
     const float* __restrict__ part, const int32_t* __restrict__ ctl, int S, int I, int SP,
-    int sf_stride, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    int sf_rows, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
     pdl_launch_dependents();
     pdl_wait();
     const int r = blockIdx.y;
     const int blk = blockIdx.x * (mxtc::PREP_THREADS / 32) + (threadIdx.x >> 5);
-    if (pad_scale_block(r, blk, I, SP, sf_stride, sf)) return;
+    if (pad_scale_block(r, blk, I, SP, sf_rows, sf)) return;
     const int i = blk * 32 + (threadIdx.x & 31);
     const int splits = ctl[0];
     float g = 0.f, u = 0.f;
@@ -631,7 +635,7 @@ __global__ void __launch_bounds__(mxtc::PREP_THREADS) mx_tc_swiglu_kernel(
         u += row[I + i];
     }
     const float h = __bfloat162float(__float2bfloat16_rn(g / (1.f + __expf(-g)) * u));
-    store_e4m3_pair(h, r, blk, I, SP, sf_stride, q, sf);
+    store_e4m3_pair(h, r, blk, I, SP, sf_rows, q, sf);
 }
 
 // GEMM 2 epilogue: y_slots[r] = routed_scale * topk_w[perm[r]] * sum over splits.
@@ -702,8 +706,10 @@ int64_t mx_tc_part_floats(int64_t slots, int H, int I) {
     return rows * cols;
 }
 
-// Activation scale rows: 4 bytes per K-group, whole K-groups.
-static int mx_tc_sf_stride(int K) { return (K + mxtc::KG - 1) / mxtc::KG * 4; }
+// 32-blocks of a row in whole K-groups (the prep kernels' grid).
+static int mx_tc_blocks(int K) { return (K + mxtc::KG - 1) / mxtc::KG * 4; }
+// Rows of an activation scale block per K-group.
+int mx_tc_sf_rows(int64_t SP) { return static_cast<int>(2 * SP + mxtc::SF_PAD_ROWS); }
 
 // The prepared weights of the tensor-core path (mx_tc_prepare), in this
 // order, each part 256-byte aligned:
@@ -899,13 +905,14 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
                        mxtc::HALF_ROWS) ||
         !make_map_e4m3(&map_x, xq, SP, s.H, CH) || !make_map_e4m3(&map_h, hq, SP, s.I, CH))
         return cudaErrorInvalidValue;
-    const int sf_x = mx_tc_sf_stride(s.H), sf_h = mx_tc_sf_stride(s.I);
+    const int nb_x = mx_tc_blocks(s.H), nb_h = mx_tc_blocks(s.I);
+    const int sf_rows = mx_tc_sf_rows(SP);
 
     constexpr int WPB = mxtc::PREP_THREADS / 32;
-    cudaError_t e = launch_pdl(mx_tc_prep_x_kernel, dim3((sf_x + WPB - 1) / WPB, S),
+    cudaError_t e = launch_pdl(mx_tc_prep_x_kernel, dim3((nb_x + WPB - 1) / WPB, S),
                                dim3(mxtc::PREP_THREADS), 0, st,
-                               static_cast<const __nv_bfloat16*>(x), perm, s.k, s.H, SP, sf_x, xq,
-                               xsf);
+                               static_cast<const __nv_bfloat16*>(x), perm, s.k, s.H, SP, sf_rows,
+                               xq, xsf);
     if (e != cudaSuccess) return e;
 
     MxTcParams p{};
@@ -922,21 +929,20 @@ static cudaError_t run_tc(const moe_shape& s, const void* x, const int32_t* offs
     p.w_scales = gu_s;
     p.w_tiled = m.tiled;
     p.act_sf = xsf;
-    p.sf_stride = sf_x;
+    p.sf_rows = sf_rows;
     p.K = s.H;
     p.wrows = 2 * static_cast<int64_t>(s.I);
     p.n_out = 2 * s.I;
     p.mtiles = s.I / mxtc::HALF_ROWS;
     e = launch_tc<0, CH, KGS, CPS, TILED>(map_gu, map_x, p, num_sms, st);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(mx_tc_swiglu_kernel, dim3((sf_h + WPB - 1) / WPB, S),
-                   dim3(mxtc::PREP_THREADS), 0, st, part, ctl, S, s.I, SP, sf_h, hq, hsf);
+    e = launch_pdl(mx_tc_swiglu_kernel, dim3((nb_h + WPB - 1) / WPB, S),
+                   dim3(mxtc::PREP_THREADS), 0, st, part, ctl, S, s.I, SP, sf_rows, hq, hsf);
     if (e != cudaSuccess) return e;
     // GEMM 2: down, K = I, 128 rows per tile (the last one partial when H % 128 != 0)
     p.w_scales = dn_s;
     p.w_tiled = m.tiled_dn;
     p.act_sf = hsf;
-    p.sf_stride = sf_h;
     p.K = s.I;
     p.wrows = s.H;
     p.n_out = s.H;

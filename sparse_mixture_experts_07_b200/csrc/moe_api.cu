@@ -47,6 +47,7 @@ int64_t mx_tc_prepared_bytes(const moe_shape&);
 cudaError_t launch_mx_tc_prepare(const moe_shape&, const uint8_t*, const uint8_t*, const uint8_t*,
                                  const uint8_t*, void*, int, cudaStream_t);
 int64_t mx_tc_plane_rows(int64_t slots);
+int mx_tc_sf_rows(int64_t SP);
 int64_t mx_tc_part_floats(int64_t slots, int H, int I);
 cudaError_t launch_ffn_decode_mxfp4_tc(const moe_shape&, const void*, const int32_t*,
                                        const int32_t*, const float*, const uint8_t*,
@@ -152,17 +153,19 @@ Workspace layout(const moe_shape& s) {
         off += align_up(static_cast<size_t>(Tk) * 4);
         if (s.H % 64 == 0 && s.I % 64 == 0) {
             // block-scaled tensor-core path: E4M3 hi/lo planes of x and h with
-            // their exponents (rows of 4 bytes per 128-column K-group), the
-            // split partials, and the split count
+            // their exponents (per 128-column K-group a block of
+            // mx_tc_sf_rows 16-byte rows), the split partials, and the split
+            // count
             const size_t SP = static_cast<size_t>(moe::mx_tc_plane_rows(Tk));
+            const size_t sf_block = static_cast<size_t>(moe::mx_tc_sf_rows(SP)) * 16;
             w.mx_xq_off = off;
             off += align_up(2 * SP * s.H);
             w.mx_xsf_off = off;
-            off += align_up(2 * SP * ((s.H + 127) / 128 * 4));
+            off += align_up((s.H + 127) / 128 * sf_block);
             w.mx_hq_off = off;
             off += align_up(2 * SP * s.I);
             w.mx_hsf_off = off;
-            off += align_up(2 * SP * ((s.I + 127) / 128 * 4));
+            off += align_up((s.I + 127) / 128 * sf_block);
             w.mx_part_off = off;
             off += align_up(static_cast<size_t>(moe::mx_tc_part_floats(Tk, s.H, s.I)) * 4);
             w.mx_ctl_off = off;
