@@ -50,11 +50,11 @@
 // its size, so the SM moves more bytes with more issuing threads.  Stages of
 // one K-group, weights as a 4D tensor-map box (the tile's two 64-row halves).
 //   warp 0     producer: lane 0 issues the TMA boxes of a stage (the weight
-//              tile, the hi and lo activation rows) and, on prepared
-//              weights, the bulk copy of the stage's weight-scale atom; all
-//              32 lanes copy the activation scale words (and, on raw
-//              weights, the weight scale words) with 4-byte cp.async and
-//              report them on the stage barrier with cp.async.mbarrier.arrive;
+//              tile, the hi and lo activation rows) and the bulk copies of
+//              the activation scales and, on prepared weights, of the
+//              stage's weight-scale atom; on raw weights all 32 lanes copy
+//              the weight scale words with 4-byte cp.async and report them
+//              on the stage barrier with cp.async.mbarrier.arrive;
 //   warp 1     allocates tensor memory; one thread copies the stage's scale
 //              factors to tensor memory and issues its four MMAs;
 //   warps 2-5  epilogue: tcgen05.ld of their 32 lanes, hi + lo, fp32 partial
