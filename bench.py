@@ -343,7 +343,8 @@ class Workload:
 
     def forward(self, stream=None):
         """The moe_forward region alone, on the plan the last step left in the buffers."""
-        moe, s, L = self.moe, self.shape, self.layer
+        moe, L = self.moe, self.layer
+        s = L.shape   # the shape the layer's calls run on (shared experts merged)
         b = L.buf
         if L.mx_prepared is not None:
             moe.forward_mxfp4_prepared(s, self.x, b["offsets"], b["perm"], b["topk_w"], self.mx,
@@ -359,7 +360,8 @@ class Workload:
 
     def step(self, stream, fwd_start=None, fwd_end=None):
         """route + permute -> forward -> combine, with events around the forward."""
-        moe, s, L = self.moe, self.shape, self.layer
+        moe, L = self.moe, self.layer
+        s = L.shape
         b = L.buf
         moe.route_permute(s, self.x, L.w_router, L.router_bias, L.workspace, L.err_flag, out=b,
                           stream=stream, w_split=L.w_split)
@@ -466,7 +468,7 @@ def measure_train(name, dev, steps, peaks) -> dict:
     import sparse_mixture_experts_07_b200 as moe
     cfg = CONFIGS[name]
     w = Workload(cfg, "bf16", dev, seed=0)
-    L, s, x = w.layer, w.shape, w.x
+    L, s, x = w.layer, w.layer.shape, w.x
     b = L.buf
     state = torch.empty(moe.train_state_size(s), dtype=torch.uint8, device=dev)
     bws = torch.empty(moe.backward_workspace_size(s), dtype=torch.uint8, device=dev)
@@ -520,7 +522,7 @@ def run_cuda(args, cfg, rank, local, world):
 
     dev = torch.device("cuda", local)
     wl = Workload(cfg, args.weights, dev, seed=rank)
-    layer, x, mx, shape = wl.layer, wl.x, wl.mx, wl.shape
+    layer, x, mx = wl.layer, wl.x, wl.mx
     stream = torch.cuda.current_stream(dev)
 
     def step():

@@ -257,6 +257,33 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const int3
                        void* y_slots, int32_t* err_flag, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* The S always-on shared experts of `shape` rearranged, once at load time,
+ * into one shared expert of intermediate size S * I_shared ("Instella-MoE
+ * modeling code walk-through", FarSkipMoE and "config at a glance": two
+ * shared experts whose outputs are added to every token; "Mixture of Experts
+ * in Transformers", WeightConverter section: layout conversions belong to
+ * weight loading).  The sum over s of down_s (SiLU(gate_s x) * up_s x) is the
+ * one expert's down (SiLU(gate x) * up x) with gate, up and h stacked along
+ * the intermediate dimension and down concatenated along its columns, so
+ * moe_forward / moe_combine called with n_shared = 1 and
+ * I_shared = S * I_shared on these arrays compute the same block with one
+ * shared slot row per token instead of S (S - 1 fewer rows of H written by
+ * the forward and read by the combine; one rounding of the shared sum
+ * instead of S).
+ *   sh_gate_up       [S, 2Is, H]  dtype input (as moe_forward)
+ *   sh_down          [S, H, Is]   dtype input
+ *   gate_up_merged   [2 S Is, H]  dtype output, caller-owned: rows
+ *                    [s Is, (s+1) Is) are expert s's gate rows, rows
+ *                    [S Is + s Is, S Is + (s+1) Is) its up rows
+ *   down_merged      [H, S Is]    dtype output, caller-owned: columns
+ *                    [s Is, (s+1) Is) are expert s's down columns
+ * Device pointers; outputs must not overlap the inputs.  Errors:
+ * MOE_ERR_INVALID_ARG for n_shared == 0 or a NULL pointer, MOE_ERR_CUDA when
+ * a copy fails to launch.  The copies are enqueued on `stream`. */
+MOE_API moe_status moe_shared_merge(const moe_shape* shape, const void* sh_gate_up,
+                                    const void* sh_down, void* gate_up_merged,
+                                    void* down_merged, void* stream);
+
 /* moe_forward with the routed experts' weights in MXFP4, for decode batches
  * ("Mixture of Experts in Transformers", section "from dense to sparse": at
  * small batch the time is the bytes of the active experts' weights, and the

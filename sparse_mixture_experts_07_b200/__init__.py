@@ -9,5 +9,5 @@ from .moe import (MOE_BF16, MOE_F32, MoEError, MoEGraph, MoELayer, Shape,  # noq
                   combine_experts, forward, forward_experts, forward_mxfp4,
                   forward_mxfp4_prepared, forward_train, mxfp4_prepare,
                   load_library, permute, route, route_noaux_tc, route_permute, router_split,
-                  train_state_size, workspace_size)
+                  shared_merge, train_state_size, workspace_size)
 from .expert_parallel import MoELayerEP, allreduce_partial, expert_range  # noqa: F401

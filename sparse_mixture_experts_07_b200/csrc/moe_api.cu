@@ -502,6 +502,36 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* off
                          static_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_shared_merge(const moe_shape* shape, const void* sh_gate_up, const void* sh_down,
+                            void* gate_up_merged, void* down_merged, void* stream) {
+    moe_status st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    const moe_shape& s = *shape;
+    if (s.n_shared == 0 || !sh_gate_up || !sh_down || !gate_up_merged || !down_merged)
+        return MOE_ERR_INVALID_ARG;
+    const size_t eb = elem_bytes(s);
+    const size_t S = static_cast<size_t>(s.n_shared), Is = static_cast<size_t>(s.I_shared);
+    const size_t H = static_cast<size_t>(s.H);
+    const size_t block = Is * H * eb;   // one expert's gate (or up) rows
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const auto* src_gu = static_cast<const uint8_t*>(sh_gate_up);
+    auto* dst_gu = static_cast<uint8_t*>(gate_up_merged);
+    for (size_t e = 0; e < S; ++e) {
+        // gate rows of expert e, then its up rows, each one contiguous block
+        if (cudaMemcpyAsync(dst_gu + e * block, src_gu + 2 * e * block, block,
+                            cudaMemcpyDeviceToDevice, cs) != cudaSuccess ||
+            cudaMemcpyAsync(dst_gu + (S + e) * block, src_gu + (2 * e + 1) * block, block,
+                            cudaMemcpyDeviceToDevice, cs) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        // expert e's [H, Is] down matrix into columns [e Is, (e+1) Is) of [H, S Is]
+        if (cudaMemcpy2DAsync(static_cast<uint8_t*>(down_merged) + e * Is * eb, S * Is * eb,
+                              static_cast<const uint8_t*>(sh_down) + e * block, Is * eb,
+                              Is * eb, H, cudaMemcpyDeviceToDevice, cs) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
 moe_status moe_forward_experts(const moe_shape* shape, int32_t e_begin, int32_t e_end,
                                const void* x, const int32_t* offsets, const int32_t* perm,
                                const float* topk_w, const void* gate_up_local,

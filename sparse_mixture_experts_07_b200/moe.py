@@ -8,7 +8,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 from typing import Optional
 
 import torch
@@ -23,7 +23,7 @@ EXPORTS = ("moe_status_str", "moe_workspace_size", "moe_route", "moe_permute", "
            "moe_combine", "moe_router_split_size", "moe_router_split", "moe_route_split",
            "moe_forward_mxfp4", "moe_forward_experts", "moe_combine_experts", "moe_cast_f32",
            "moe_route_noaux_tc", "moe_train_state_size", "moe_forward_train",
-           "moe_backward_workspace_size", "moe_backward")
+           "moe_backward_workspace_size", "moe_backward", "moe_shared_merge")
 
 
 class MoEShape(ctypes.Structure):
@@ -66,6 +66,7 @@ def load_library(path: str = LIB_PATH):
                                                ctypes.c_size_t, P]
     lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_combine.argtypes = [S, P, P, P, P]
+    lib.moe_shared_merge.argtypes = [S, P, P, P, P, P]
     lib.moe_router_split_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
     lib.moe_router_split.argtypes = [S, P, P, ctypes.c_size_t, P]
     lib.moe_route_split.argtypes = [S, P, P, P, P, P, P, P, P, P]
@@ -256,6 +257,21 @@ def forward(shape: Shape, x, offsets, perm, topk_w, gate_up, down, sh_gate_up, s
     return y_slots
 
 
+def shared_merge(shape: Shape, sh_gate_up, sh_down, stream=None):
+    """The shape's S shared experts as one of width S * I_shared (moe_shared_merge),
+    done once at load time: (merged_shape, gate_up [1, 2 S Is, H], down [1, H, S Is])."""
+    lib = load_library()
+    S, Is, H = shape.n_shared, shape.I_shared, shape.H
+    if sh_gate_up.shape != (S, 2 * Is, H) or sh_down.shape != (S, H, Is) \
+            or not (sh_gate_up.is_contiguous() and sh_down.is_contiguous()):
+        raise ValueError("shared experts must be contiguous [S, 2Is, H] and [S, H, Is]")
+    gu = torch.empty(1, 2 * S * Is, H, dtype=shape.torch_dtype, device=sh_gate_up.device)
+    dn = torch.empty(1, H, S * Is, dtype=shape.torch_dtype, device=sh_gate_up.device)
+    _check(lib.moe_shared_merge(ctypes.byref(shape.c()), _ptr(sh_gate_up), _ptr(sh_down),
+                                _ptr(gu), _ptr(dn), _stream(stream)), "moe_shared_merge")
+    return replace(shape, n_shared=1, I_shared=S * Is), gu, dn
+
+
 def forward_mxfp4(shape: Shape, x, offsets, perm, topk_w, mxfp4: dict, workspace, err_flag,
                   y_slots=None, stream=None):
     """moe_forward with MXFP4 routed-expert weights (decode batches, T <= 64):
@@ -422,16 +438,22 @@ class MoELayer:
 
     Holds the weights (device tensors) and a reusable workspace; `__call__`
     takes x [T, H] on the device and returns y [T, H].  Intermediates of the
-    last call are kept in `self.last` for inspection.
+    last call are kept in `self.last` for inspection.  Two or more shared
+    experts are merged at construction into one of their summed width
+    (moe_shared_merge): `self.shape` and `self.sh_gate_up` / `self.sh_down`
+    are then the merged ones the library calls run on, and y_slots holds one
+    shared row per token.
     """
 
     def __init__(self, shape: Shape, w_router, router_bias, gate_up=None, down=None,
-                 sh_gate_up=None, sh_down=None, mxfp4=None, routing=None):
+                 sh_gate_up=None, sh_down=None, mxfp4=None, routing=None, merge_shared=True):
         """Expert weights either as gate_up / down (dtype of `shape`), or as
         `mxfp4` = {gate_up_q, gate_up_s, down_q, down_s} (decode batches).
         `routing`: None for top-k with a softmax over the selected k (the bias
         added to the logits), or ("noaux_tc", n_group, topk_group) for
-        DeepSeek-V3 routing (the bias steers the selection only)."""
+        DeepSeek-V3 routing (the bias steers the selection only).
+        `merge_shared`: run two or more shared experts as one (the default) or
+        as separate groups."""
         self.shape = shape
         self.mxfp4 = mxfp4
         self.routing = routing
@@ -442,6 +464,9 @@ class MoELayer:
         self.w_split = router_split(shape, w_router)
         self.gate_up, self.down = gate_up, down
         self.sh_gate_up, self.sh_down = sh_gate_up, sh_down
+        if merge_shared and shape.n_shared > 1 and mxfp4 is None:
+            shape, self.sh_gate_up, self.sh_down = shared_merge(shape, sh_gate_up, sh_down)
+            self.shape = shape
         # MXFP4 weights prepared once for the tensor-core kernel where it
         # takes the shape (decode batches, H and I multiples of 64)
         self.mx_prepared = None

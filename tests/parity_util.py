@@ -74,11 +74,14 @@ def to_device(inp: dict, dev="cuda") -> dict:
     return out
 
 
-def run_gpu(cfg: MoEConfig, dinp: dict) -> dict:
-    """Every step through the C ABI; returns host copies of all outputs."""
+def run_gpu(cfg: MoEConfig, dinp: dict, merge_shared: bool = True) -> dict:
+    """Every step through the C ABI; returns host copies of all outputs.
+    `merge_shared`: two or more shared experts run as one merged expert (the
+    layer's default) or as separate groups."""
     shape = moe.Shape.from_config(cfg)
     layer = moe.MoELayer(shape, dinp["w_router"], dinp["router_bias"], dinp["gate_up"],
-                         dinp["down"], dinp["sh_gate_up"], dinp["sh_down"])
+                         dinp["down"], dinp["sh_gate_up"], dinp["sh_down"],
+                         merge_shared=merge_shared)
     # logits of the router that splits the weight in every CTA, and of the
     # router on the weight split at load time (the layer's path)
     idx, w, logits = moe.route(shape, dinp["x"], dinp["w_router"], dinp["router_bias"],

@@ -140,6 +140,23 @@ def test_router_split_size_zero_where_the_tensor_core_router_does_not_apply(lib)
     assert _split_size(lib, _shape(k=0))[0] == 1
 
 
+def test_shared_merge_argument_checks(lib):
+    """moe_shared_merge rejects a shape without shared experts, NULL pointers
+    and invalid shapes before any copy is enqueued."""
+    p = ctypes.c_void_p(4096)
+    s = _shape(n_shared=2, I_shared=64)
+    args = [p, p, p, p]
+    for i in range(4):
+        a = list(args)
+        a[i] = None
+        assert lib.moe_shared_merge(ctypes.byref(s), *a, None) == 1
+    none = _shape(n_shared=0, I_shared=0)
+    assert lib.moe_shared_merge(ctypes.byref(none), *args, None) == 1
+    assert lib.moe_shared_merge(ctypes.byref(_shape(n_shared=2, I_shared=0)), *args, None) == 1
+    assert lib.moe_shared_merge(ctypes.byref(_shape(n_shared=2, I_shared=60)), *args, None) == 2
+    assert lib.moe_shared_merge(None, *args, None) == 1
+
+
 def test_router_split_argument_checks(lib):
     s = _shape(E=8, H=128)
     _, need = _split_size(lib, s)

@@ -36,8 +36,9 @@ def _run(cfg, inp, dy, aux_coef=0.0):
     import sparse_mixture_experts_07_b200 as moe
     d = to_device(inp)
     shape = moe.Shape.from_config(cfg)
+    # the layer only supplies buffers here: keep its shared experts as given
     layer = moe.MoELayer(shape, d["w_router"], d["router_bias"], d["gate_up"], d["down"],
-                         d["sh_gate_up"], d["sh_down"])
+                         d["sh_gate_up"], d["sh_down"], merge_shared=False)
     b = layer.buf
     idx, w, logits = moe.route(shape, d["x"], d["w_router"], d["router_bias"], out=b,
                                logits=True, err_flag=layer.err_flag, w_split=layer.w_split)

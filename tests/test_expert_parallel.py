@@ -112,8 +112,9 @@ def test_emulated_ranks_match_the_oracle_and_one_rank(cuda_ok, cfg, world):
     inp = make_inputs(cfg, seed=0)
     d = to_device(inp)
     shape = moe.Shape.from_config(cfg)
+    # shared experts as separate groups, like the ranks' layers (slot rows compared)
     full = moe.MoELayer(shape, d["w_router"], d["router_bias"], d["gate_up"], d["down"],
-                        d["sh_gate_up"], d["sh_down"])
+                        d["sh_gate_up"], d["sh_down"], merge_shared=False)
     y_full = full(d["x"]).clone()
     slots_full = full.last["y_slots"].clone()
     offsets = full.last["offsets"].cpu().numpy()

@@ -70,6 +70,48 @@ def test_small_configs(cuda_ok, cfg):
     check_outputs(cfg, inp, res)
 
 
+SHARED = [c for c in SMALL if c.n_shared > 1]
+
+
+@pytest.mark.parametrize("cfg", SHARED, ids=lambda c: c.name)
+def test_shared_experts_merged_and_separate(cuda_ok, cfg):
+    """Two shared experts run as one merged expert (the layer's default) and as
+    separate groups: both match the oracle, whose shared experts stay
+    separate; the routed slot rows are the same bits either way."""
+    inp = make_inputs(cfg, seed=0, weights_device="cpu")
+    d = to_device(inp)
+    merged = run_gpu(cfg, d)
+    separate = run_gpu(cfg, d, merge_shared=False)
+    tk = cfg.T * cfg.k
+    assert merged["y_slots"].shape[0] == cfg.T * (cfg.k + 1)
+    assert separate["y_slots"].shape[0] == cfg.T * (cfg.k + cfg.n_shared)
+    assert torch.equal(merged["y_slots"][:tk], separate["y_slots"][:tk])
+    for res in (merged, separate):
+        assert res["err"] == 0
+        check_routing(cfg, inp, res)
+        check_outputs(cfg, inp, res)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_shared_merge_layout(cuda_ok, dtype):
+    """moe_shared_merge stacks the experts' gate rows, then their up rows, and
+    concatenates their down matrices along the columns."""
+    import sparse_mixture_experts_07_b200 as moe
+    S, Is, H = 3, 40, 24
+    shape = moe.Shape(T=4, H=H, I=16, E=4, k=2, n_shared=S, I_shared=Is,
+                      dtype=moe.MOE_BF16 if dtype == "bf16" else moe.MOE_F32)
+    g = torch.Generator().manual_seed(1)
+    gu = torch.randn(S, 2 * Is, H, generator=g).to(shape.torch_dtype)
+    dn = torch.randn(S, H, Is, generator=g).to(shape.torch_dtype)
+    m_shape, m_gu, m_dn = moe.shared_merge(shape, gu.cuda(), dn.cuda())
+    torch.cuda.synchronize()
+    assert (m_shape.n_shared, m_shape.I_shared) == (1, S * Is)
+    want_gu = torch.cat([gu[:, :Is].reshape(S * Is, H), gu[:, Is:].reshape(S * Is, H)])
+    want_dn = torch.cat([dn[e] for e in range(S)], dim=1)
+    assert torch.equal(m_gu.cpu()[0], want_gu)
+    assert torch.equal(m_dn.cpu()[0], want_dn)
+
+
 def test_routed_slot_rows_hold_weighted_expert_outputs(cuda_ok):
     # y_slots row p = routed_scale * w * FFN_e(x_t) for slot perm[p]
     import oracle
@@ -142,6 +184,21 @@ def test_full_size_sampled(cuda_ok, name):
         # every routed expert with slots has at least one checked row
         hit = np.unique(o_idx[toks].reshape(-1))
         assert np.array_equal(hit, np.nonzero(np.diff(o_offsets))[0])
+    check_outputs(cfg, host, res, tokens=toks)
+
+
+def test_full_size_shared_experts_separate(cuda_ok):
+    """The DeepSeek-V3-shaped layer with its two shared experts run as separate
+    groups (the full-size test above runs them merged): a stratified sample of
+    tokens against the oracle."""
+    cfg = CONFIGS["dsv3"]
+    inp = make_inputs(cfg, seed=0, weights_device="cuda")
+    res = run_gpu(cfg, to_device(inp), merge_shared=False)
+    assert res["err"] == 0
+    assert res["y_slots"].shape[0] == cfg.T * (cfg.k + cfg.n_shared)
+    host = {key: (v.cpu() if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
+    o_idx, _, o_offsets, o_perm = check_routing(cfg, host, res)
+    toks = stratified_tokens(o_idx, o_offsets, o_perm, 512)
     check_outputs(cfg, host, res, tokens=toks)
 
 
