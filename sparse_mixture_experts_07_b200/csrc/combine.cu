@@ -91,13 +91,22 @@ __global__ void __launch_bounds__(256) combine_bf16_pipelined_kernel(
             float acc[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-            for (int j = 0; j < nrows; ++j) {
-                const uint4 u = y_slots[rows_sh[buf][j] * vec_per_row + v];
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            // up to four rows' loads in flight at once, summed in row order
+            for (int j = 0; j < nrows; j += 4) {
+                const int n = nrows - j < 4 ? nrows - j : 4;
+                uint4 u[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    acc[2 * q] += bf16_to_f32(static_cast<uint16_t>(w[q] & 0xffffu));
-                    acc[2 * q + 1] += bf16_to_f32(static_cast<uint16_t>(w[q] >> 16));
+                for (int r = 0; r < 4; ++r)
+                    if (r < n) u[r] = y_slots[rows_sh[buf][j + r] * vec_per_row + v];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r >= n) break;
+                    const uint32_t w[4] = {u[r].x, u[r].y, u[r].z, u[r].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[2 * q] += bf16_to_f32(static_cast<uint16_t>(w[q] & 0xffffu));
+                        acc[2 * q + 1] += bf16_to_f32(static_cast<uint16_t>(w[q] >> 16));
+                    }
                 }
             }
             uint4 o;
@@ -114,10 +123,21 @@ __global__ void __launch_bounds__(256) combine_bf16_pipelined_kernel(
 cudaError_t launch_combine(const moe_shape& s, const void* y_slots, const int32_t* inv, void* y,
                            cudaStream_t st) {
     if (s.dtype == MOE_BF16) {
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess)
+        // as many CTAs as are resident at once, so that every CTA starts
+        // right away (looked up once per device)
+        static int resident[64] = {0};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+        if (resident[dev] <= 0) {
+            int sms = 148, per_sm = 0;
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int64_t cap = static_cast<int64_t>(sms) * 8;    // 8 CTAs of 256 threads per SM
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &per_sm, combine_bf16_pipelined_kernel, 256, 0) != cudaSuccess ||
+                per_sm <= 0)
+                per_sm = 4;
+            resident[dev] = sms * per_sm;
+        }
+        const int64_t cap = resident[dev];
         const unsigned grid = static_cast<unsigned>(s.T < cap ? s.T : cap);
         return launch_pdl(combine_bf16_pipelined_kernel, dim3(grid), dim3(256), 0, st,
                           static_cast<const uint4*>(y_slots), inv, static_cast<uint4*>(y), s.T,
