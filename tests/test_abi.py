@@ -157,6 +157,21 @@ def test_shared_merge_argument_checks(lib):
     assert lib.moe_shared_merge(None, *args, None) == 1
 
 
+def test_shared_merge_binding_checks_shapes(lib):
+    """The binding rejects shared-expert tensors of the wrong shape or layout
+    before it calls the library."""
+    import torch
+    shape = moe.Shape(T=4, H=16, I=8, E=4, k=2, n_shared=2, I_shared=8)
+    gu = torch.zeros(2, 16, 16, dtype=torch.bfloat16)
+    dn = torch.zeros(2, 16, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        moe.shared_merge(shape, gu[:, :8], dn)
+    with pytest.raises(ValueError):
+        moe.shared_merge(shape, gu, dn.transpose(1, 2).contiguous())
+    with pytest.raises(ValueError):
+        moe.shared_merge(shape, gu, torch.zeros(2, 8, 16, dtype=torch.bfloat16).transpose(1, 2))
+
+
 def test_router_split_argument_checks(lib):
     s = _shape(E=8, H=128)
     _, need = _split_size(lib, s)
