@@ -166,12 +166,27 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           uint4* __restrict__ x_perm, int64_t n_rows,
                                                           int vec_per_row, int k) {
     const int64_t total = n_rows * vec_per_row;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * 256) {
-        const int64_t p = i / vec_per_row;
-        const int v = static_cast<int>(i - p * vec_per_row);
-        const int64_t q = perm[p];
-        if (q >= 0 && q < n_rows) x_perm[i] = x[(q / k) * vec_per_row + v];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+    // four pieces per thread and pass, their loads in flight together
+    for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i0 < total;
+         i0 += 4 * stride) {
+        uint4 val[4];
+        bool ok[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t i = i0 + u * stride;
+            ok[u] = false;
+            if (i < total) {
+                const int64_t p = i / vec_per_row;
+                const int v = static_cast<int>(i - p * vec_per_row);
+                const int64_t q = perm[p];
+                ok[u] = q >= 0 && q < n_rows;
+                if (ok[u]) val[u] = x[(q / k) * vec_per_row + v];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (ok[u]) x_perm[i0 + u * stride] = val[u];
     }
 }
 
@@ -195,14 +210,24 @@ __global__ void __launch_bounds__(256) gather_by_token_kernel(const uint4* __res
                                                               int64_t n_tokens, int vec_per_row,
                                                               int k) {
     const int64_t total = n_tokens * vec_per_row;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * 256) {
-        const int64_t t = i / vec_per_row;
-        const int v = static_cast<int>(i - t * vec_per_row);
-        const uint4 val = x[i];
-        for (int j = 0; j < k; ++j) {
-            const int64_t p = inv[t * k + j];
-            if (p >= 0 && p < n_tokens * k) x_perm[p * vec_per_row + v] = val;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+    // four pieces per thread and pass, their loads in flight together
+    for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i0 < total;
+         i0 += 4 * stride) {
+        uint4 val[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u * stride < total) val[u] = x[i0 + u * stride];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i >= total) break;
+            const int64_t t = i / vec_per_row;
+            const int v = static_cast<int>(i - t * vec_per_row);
+            for (int j = 0; j < k; ++j) {
+                const int64_t p = inv[t * k + j];
+                if (p >= 0 && p < n_tokens * k) x_perm[p * vec_per_row + v] = val[u];
+            }
         }
     }
 }
