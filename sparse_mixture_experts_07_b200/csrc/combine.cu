@@ -7,9 +7,11 @@
 // GraniteMoeSWA decoder layer, moe output + shared_mlp).  The sum is float32 in
 // a fixed order (j ascending, then s ascending) and is rounded once.
 //
-// One CTA of 256 threads per token row; each thread owns 16-byte vectors of
-// the row, so every y_slots row is read once, coalesced.  Memory-bound:
-// (k + S) * H * elem bytes read and H * elem bytes written per token.
+// float32: one CTA of 256 threads per token row, each thread owning 16-byte
+// vectors (or single elements when H % 4 != 0) of the row, so every y_slots
+// row is read once, coalesced; bf16: the persistent kernel further down.
+// Memory-bound: (k + S) * H * elem bytes read and H * elem bytes written per
+// token.
 #include "common.cuh"
 
 namespace moe {
@@ -30,15 +32,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_sl
             for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
             for (int j = 0; j < k + S; ++j) {
                 const T* src = y_slots + rows[j] * H + c;
-                if constexpr (VEC == 8) {
-                    const uint4 u = *reinterpret_cast<const uint4*>(src);
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        acc[2 * v] += bf16_to_f32(static_cast<uint16_t>(w[v] & 0xffffu));
-                        acc[2 * v + 1] += bf16_to_f32(static_cast<uint16_t>(w[v] >> 16));
-                    }
-                } else if constexpr (VEC == 4) {
+                if constexpr (VEC == 4) {
                     const float4 u = *reinterpret_cast<const float4*>(src);
                     acc[0] += u.x; acc[1] += u.y; acc[2] += u.z; acc[3] += u.w;
                 } else {
@@ -47,14 +41,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_sl
                 }
             }
             T* dst = y + t * H + c;
-            if constexpr (VEC == 8) {
-                uint4 u;
-                u.x = pack_bf16x2(acc[0], acc[1]);
-                u.y = pack_bf16x2(acc[2], acc[3]);
-                u.z = pack_bf16x2(acc[4], acc[5]);
-                u.w = pack_bf16x2(acc[6], acc[7]);
-                *reinterpret_cast<uint4*>(dst) = u;
-            } else if constexpr (VEC == 4) {
+            if constexpr (VEC == 4) {
                 *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             } else {
 #pragma unroll
@@ -144,11 +131,7 @@ cudaError_t launch_combine(const moe_shape& s, const void* y_slots, const int32_
                           s.H / 8, s.k, s.n_shared);
     }
     const unsigned grid = static_cast<unsigned>(s.T < 1048576 ? s.T : 1048576);
-    if (s.dtype == MOE_BF16) {
-        combine_kernel<__nv_bfloat16, 8><<<grid, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(y_slots), inv, static_cast<__nv_bfloat16*>(y), s.T,
-            s.H, s.k, s.n_shared);
-    } else if (s.H % 4 == 0) {
+    if (s.H % 4 == 0) {
         combine_kernel<float, 4><<<grid, 256, 0, st>>>(static_cast<const float*>(y_slots), inv,
                                                        static_cast<float*>(y), s.T, s.H, s.k,
                                                        s.n_shared);
